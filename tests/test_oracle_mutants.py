@@ -1,0 +1,64 @@
+"""Plant plausible mistakes in copies of the oracle and check the pins catch each.
+
+Every mutant is a one-line edit of oracle/jl_oracle.c (a wrong comparison, a
+dropped term, a flipped sign, a wrong index), compiled on the CPU into a
+temporary library.  The real oracle is never modified.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle_pins
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "jl_oracle.c")
+
+MUTANTS = {
+    "local_boundary_inclusive": ("return (q - k) < w_local;", "return (q - k) <= w_local;"),
+    "remap_ceil": ("long long jlo_remap(long long x, long long G) { return x / G; }",
+                   "long long jlo_remap(long long x, long long G) { return (x + G - 1) / G; }"),
+    "group_size_floor": ("long long g = (L + w_pretrained - 1) / w_pretrained;",
+                         "long long g = L / w_pretrained;"),
+    "rope_sin_sign": ("y[i] = x1 * c - x2 * s;", "y[i] = x1 * c + x2 * s;"),
+    "rope_second_half": ("y[i + h] = x1 * s + x2 * c;", "y[i + h] = x2 * s + x1 * c;"),
+    "theta_exponent": ("pow(base, -2.0 * (double)i / (double)D)",
+                       "pow(base, -1.0 * (double)i / (double)D)"),
+    "lse_drops_max": ("return M + log(Z);", "return log(Z);"),
+    "remote_uses_standard_query": ("s[kk] = scale * jlo_dot(qr, krem + kk * D, D);",
+                                   "s[kk] = scale * jlo_dot(qs, krem + kk * D, D);"),
+    "remote_uses_standard_key": ("jlo_rope(raw, krem + kk * D, D, (double)jlo_remap(kk, G), rope_base);",
+                                 "jlo_rope(raw, krem + kk * D, D, (double)kk, rope_base);"),
+    "drops_diagonal_key": ("for (long long kk = 0; kk <= qp; ++kk) {",
+                           "for (long long kk = 0; kk < qp; ++kk) {"),
+    "gqa_head_map": ("if (row_b[r] != b || row_h[r] / group != hk) continue;",
+                     "if (row_b[r] != b || row_h[r] % Hkv != hk) continue;"),
+    "decode_dq_sign": ("const double dq = (double)(jlo_remap(pos, G) - pos);",
+                       "const double dq = (double)(pos - jlo_remap(pos, G));"),
+    "decode_corrects_local_keys": ("if (jlo_is_local(pos, kk, w_local)) {\n          for (int d = 0; d < D; ++d) kc[kk * D + d] = raw[d];",
+                                   "if (0) {\n          for (int d = 0; d < D; ++d) kc[kk * D + d] = raw[d];"),
+    "decode_dk_from_position": ("const double dk = (double)(jlo_remap(kk, G) - kk);",
+                                "const double dk = (double)(jlo_remap(kk, G));"),
+    "softmax_normaliser": ("for (int d = 0; d < D; ++d) out[d] /= Z;",
+                           "for (int d = 0; d < D; ++d) out[d] /= (Z + 1.0);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path, oracle_mod):
+    before, after = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(before) == 1, f"mutation site for {name} not found exactly once"
+    mpath = tmp_path / f"{name}.c"
+    mpath.write_text(src.replace(before, after))
+    lib = tmp_path / f"lib_{name}.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                    str(mpath), "-o", str(lib), "-lm"], check=True)
+    orc = oracle_mod.Oracle(str(lib))
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except (AssertionError, ValueError, FloatingPointError):
+            caught.append(pin.__name__)
+    assert caught, f"mutant {name} passed every pin"
