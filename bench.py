@@ -1,0 +1,457 @@
+"""Benchmark of the bifocal RoPE attention hot path on B200.
+
+One step = one pass of the whole hot path on one GPU:
+  * bifocal prefill of a Qwen3-8B-shaped attention layer at L = 131072
+    (B=1, Hq=32, Hkv=8, D=128, w_pretrained=32768 -> G=4, w_local=2048,
+    rope_base=1e6, bf16 inputs N(0,1)*0.5), and
+  * bifocal single-token decode over a 131072-token cache of the same shape
+    (pos = 131071, G = 4).
+`value` is the prefill's effective TFLOP/s (4*B*Hq*D*L(L+1)/2 FLOPs per call,
+one causal QK^T + PV pass) summed over ranks / the slowest rank's time; the
+decode's KV-read GB/s is reported beside it.  Inputs (>= 268 MB each) are
+larger than the 126 MB L2, so no flush is needed between iterations.
+
+Multi-GPU (--gpus N under torchrun): every rank runs the same independent
+problem on its own GPU (weak scaling); there is no data-path collective, only
+a barrier and a max-reduction of the timings.
+
+--impl reference times the fp64 CPU oracle (the checker) on a bounded sample
+of the same workload, on rank 0 only.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_attention_bifocal_b200 import workloads as W  # noqa: E402
+
+METRIC = "bifocal prefill TFLOP/s & % bf16 peak; decode KV-read GB/s & % HBM"
+PREFILL_CFG = "qwen3_8b_L131072"
+DECODE_CFG = "qwen3_8b_decode_n131072"
+
+
+def prefill_flops(B, Hq, D, L):
+    return 4.0 * B * Hq * D * L * (L + 1) / 2
+
+
+def rows_flops(D, rows_q):
+    return float(sum(4.0 * D * (int(q) + 1) for q in rows_q))
+
+
+def kv_bytes(B, Hkv, D, n):
+    return float(B) * n * Hkv * D * 2 * 2
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return (float(p["hbm_gbs"]), float(p["bf16_tflops"]),
+                float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured")
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="jl_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    """Largest x over all ranks (the slowest rank's time)."""
+    if world == 1:
+        return x
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(seed, rank):
+    """Seed of rank's independent problem (weak scaling: one problem per GPU)."""
+    return seed + 1000 * rank
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def run_cuda(args):
+    import long_context_attention_bifocal_b200 as jl
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pc = W.PREFILL[PREFILL_CFG]
+    dc = W.DECODE[DECODE_CFG]
+    B, L, Hq, Hkv, D = pc["B"], pc["L"], pc["Hq"], pc["Hkv"], pc["D"]
+    kwp = dict(w_local=pc["w_local"], w_pretrained=pc["w_pretrained"], rope_base=pc["rope_base"])
+    n = dc["n"]
+    pos = n - 1
+    kwd = dict(w_local=dc["w_local"], w_pretrained=dc["w_pretrained"], rope_base=dc["rope_base"])
+
+    # host inputs (pinned), one independent problem per rank
+    q_h, k_h, v_h = W.prefill_inputs(B, L, Hq, Hkv, D, value_scale=pc["value_scale"],
+                                     seed=rank_seed(pc["seed"], rank))
+    qd_h, kc_h, vc_h = W.decode_inputs(dc["B"], dc["Hq"], dc["Hkv"], dc["D"], n,
+                                       seed=rank_seed(dc["seed"], rank))
+    host = [t.pin_memory() for t in (q_h, k_h, v_h, qd_h, kc_h, vc_h)]
+    q_h, k_h, v_h, qd_h, kc_h, vc_h = host
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    qd, kc, vc = qd_h.to(dev), kc_h.to(dev), vc_h.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    outd = torch.empty_like(qd)
+    lsed = torch.empty((dc["B"], dc["Hq"]), dtype=torch.float32, device=dev)
+    wsd = torch.empty(jl.decode_workspace_size(dc["B"], dc["Hq"], dc["Hkv"], dc["D"], pos),
+                      dtype=torch.uint8, device=dev)
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    outd_h = torch.empty(outd.shape, dtype=outd.dtype, pin_memory=True)
+    lsed_h = torch.empty(lsed.shape, dtype=lsed.dtype, pin_memory=True)
+    stream = torch.cuda.current_stream(dev)
+
+    def prefill(flags=0):
+        jl.bifocal_prefill(q, k, v, out=out, lse=lse, flags=flags, **kwp)
+
+    def decode(flags=0):
+        jl.bifocal_decode(qd, kc, vc, pos, out=outd, lse=lsed, workspace=wsd, flags=flags, **kwd)
+
+    # ---------------- warm-up ----------------
+    for _ in range(args.warmup):
+        prefill()
+        decode()
+    jl.check_device_status()
+    barrier(world)
+
+    # ---------------- timed region (device clock, CUDA events) ----------------
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(args.steps):
+        ev[s][0].record(stream)
+        prefill()
+        ev[s][1].record(stream)
+        decode()
+        ev[s][2].record(stream)
+    t1.record(stream)
+    barrier(world)
+    clocks = sampler.stop()
+    jl.check_device_status()
+    total_ms = t0.elapsed_time(t1)
+    pre_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
+    dec_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(args.steps)]
+    total_ms = max_over_ranks(total_ms, world)
+    pre_sum = max_over_ranks(sum(pre_ms), world)
+    dec_sum = max_over_ranks(sum(dec_ms), world)
+    launches = 4 * args.steps  # per step: key rotation + prefill, decode split + combine
+
+    # ---------------- overhead vs the same kernels without the bifocal rule ----
+    def avg_ms(fn, reps):
+        es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        for a, b in es:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return sorted(a.elapsed_time(b) for a, b in es)[reps // 2]
+
+    dec_bif = avg_ms(lambda: decode(0), 50)
+    dec_plain = avg_ms(lambda: decode(jl.NO_BIFOCAL), 50)
+    pre_plain = avg_ms(lambda: prefill(jl.NO_BIFOCAL), max(1, min(3, args.steps)))
+    pre_bif = avg_ms(lambda: prefill(0), max(1, min(3, args.steps)))
+    jl.check_device_status()
+
+    # ---------------- end to end through the public API, host buffers ----------
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e_steps = max(1, min(args.steps, 3))
+    e0.record(stream)
+    for _ in range(e_steps):
+        q.copy_(q_h, non_blocking=True)
+        k.copy_(k_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        prefill()
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        qd.copy_(qd_h, non_blocking=True)
+        kc.copy_(kc_h, non_blocking=True)
+        vc.copy_(vc_h, non_blocking=True)
+        decode()
+        outd_h.copy_(outd, non_blocking=True)
+        lsed_h.copy_(lsed, non_blocking=True)
+    e1.record(stream)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, qd_h, kc_h, vc_h))
+    d2h = sum(t.numel() * t.element_size() for t in (out_h, lse_h, outd_h, lsed_h))
+
+    flops = prefill_flops(B, Hq, D, L)
+    kvb = kv_bytes(dc["B"], dc["Hkv"], dc["D"], n)
+    value = flops * args.steps * world / (pre_sum / 1e3) / 1e12
+    dec_gbs = kvb * args.steps * world / (dec_sum / 1e3) / 1e9
+    hbm, bf16_burst, bf16_sust, src = peaks()
+    pre_launch_ms = pre_sum / args.steps
+    achieved = flops / (pre_launch_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": "qwen3_8b attention layer: bifocal prefill L=131072 + decode n=131072",
+            "prefill": {"B": B, "L": L, "Hq": Hq, "Hkv": Hkv, "D": D, **kwp, "G": 4,
+                        "values": "N(0,1)*0.5 bf16, seeded"},
+            "decode": {"B": dc["B"], "pos": pos, "Hq": dc["Hq"], "Hkv": dc["Hkv"], "D": dc["D"],
+                       **kwd, "G": 4, "values": "N(0,1) bf16, seeded"},
+            "l2": "inputs larger than L2 (Q 1 GiB, K/V 256 MiB each, KV cache 512 MiB)",
+            "parallelism": f"independent problem per GPU x{world}",
+        },
+        "decode": {
+            "value": round(dec_gbs, 1), "unit": "GB/s",
+            "us_per_call": round(dec_sum / args.steps * 1e3, 2),
+            "frac_hbm": round(dec_gbs / world / hbm, 4),
+            "overhead_vs_no_bifocal": round(dec_bif / dec_plain - 1.0, 4),
+        },
+        "prefill": {
+            "ms_per_call": round(pre_launch_ms, 3),
+            "frac_bf16_sustained": round(achieved / bf16_sust, 4),
+            "frac_bf16_burst": round(achieved / bf16_burst, 4),
+            "overhead_vs_no_bifocal": round(pre_bif / pre_plain - 1.0, 4),
+        },
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "bifocal_prefill_sm100_kernel (+ key-rotation pass, timed together)",
+            "achieved": round(achieved, 2),
+            "peak": bf16_sust,
+            "peak_kind": f"bf16 dense, sustained, {src}",
+            "unit": "TFLOP/s",
+            "frac": round(achieved / bf16_sust, 4),
+            "traffic": None,
+        },
+        "e2e": {
+            "value": round(flops * e_steps * world / (e2e_ms / 1e3) / 1e12, 2),
+            "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h),
+        },
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(q_h, k_h, v_h, qd_h, kc_h, vc_h, kwp, kwd, pos,
+                                            budget_s=args.cpu_seconds)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(q_h, k_h, v_h, qd_h, kc_h, vc_h, kwp, kwd, pos, budget_s=20.0, rows=None):
+    """The fp64 oracle, as it stands, on a bounded sample of the same workload:
+    a few seeded rows per query head of the prefill (effective TFLOP/s over the
+    sampled rows) and the full decode (KV GB/s)."""
+    import oracle
+    orc = oracle.default()
+    B, L, Hq, D = q_h.shape
+    qa, ka, va = W.to_oracle_array(q_h), W.to_oracle_array(k_h), W.to_oracle_array(v_h)
+    per_head = rows or 8
+    rb, rq, rh = W.sample_rows(B, L, Hq, per_head=per_head, seed=123)
+    t = time.perf_counter()
+    orc.bifocal_rows(qa, ka, va, rb, rq, rh, **kwp)
+    dt = time.perf_counter() - t
+    fl = rows_flops(D, rq)
+    t = time.perf_counter()
+    orc.bifocal_decode(W.to_oracle_array(qd_h), W.to_oracle_array(kc_h[:, :pos + 1]),
+                       W.to_oracle_array(vc_h[:, :pos + 1]), pos, **kwd)
+    ddt = time.perf_counter() - t
+    kvb = kv_bytes(kc_h.shape[0], kc_h.shape[2], kc_h.shape[3], pos + 1)
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": orc.num_threads(),
+            "kind": "oracle",
+            "sample": f"prefill: {per_head} seeded rows per query head ({len(rq)} rows) of the "
+                      f"L=131072 workload, {dt:.1f} s; decode: the full n=131072 call, "
+                      f"{ddt:.1f} s ({kvb / ddt / 1e9:.3f} GB/s)"}
+
+
+def run_reference(args):
+    """The oracle arm: rank 0 only, bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import oracle
+    orc = oracle.default()
+    pc = W.PREFILL[PREFILL_CFG]
+    B, L, Hq, Hkv, D = pc["B"], pc["L"], pc["Hq"], pc["Hkv"], pc["D"]
+    kwp = dict(w_local=pc["w_local"], w_pretrained=pc["w_pretrained"], rope_base=pc["rope_base"])
+    q, k, v = W.prefill_inputs(B, L, Hq, Hkv, D, value_scale=pc["value_scale"], seed=pc["seed"])
+    qa, ka, va = W.to_oracle_array(q), W.to_oracle_array(k), W.to_oracle_array(v)
+    per_head = 2
+    times, flops = [], []
+    for s in range(args.warmup + args.steps):
+        rb, rq, rh = W.sample_rows(B, L, Hq, per_head=per_head, seed=1000 + s)
+        t = time.perf_counter()
+        orc.bifocal_rows(qa, ka, va, rb, rq, rh, **kwp)
+        dt = time.perf_counter() - t
+        if s >= args.warmup:
+            times.append(dt)
+            flops.append(rows_flops(D, rq))
+    value = sum(flops) / sum(times) / 1e12
+    sample = (f"{per_head} seeded rows per query head ({Hq * per_head} rows) of the L=131072 "
+              "prefill per step")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sum(times) / len(times), 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "qwen3_8b attention layer: bifocal prefill L=131072 (row sample)",
+                   "parallelism": "CPU oracle, rank 0"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
+                         "cores": orc.num_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+CASES = {
+    # small cases for ncu captures: inputs larger than L2, a few hundred MB on the device
+    "prefill_L32768": dict(kind="prefill", B=1, L=32768, Hq=32, Hkv=8, w_pretrained=8192),
+    "decode_n131072": dict(kind="decode", n=131072),
+}
+
+
+def run_case(args):
+    """One kernel family on a small case (warm-up + steps), for profiling."""
+    import long_context_attention_bifocal_b200 as jl
+    c = CASES[args.case]
+    dev = torch.device("cuda", 0)
+    if c["kind"] == "prefill":
+        q, k, v = W.prefill_inputs(c["B"], c["L"], c["Hq"], c["Hkv"], 128, seed=5)
+        q, k, v = q.to(dev), k.to(dev), v.to(dev)
+        kw = dict(w_local=2048, w_pretrained=c["w_pretrained"], rope_base=1e6)
+        fn = lambda: jl.bifocal_prefill(q, k, v, **kw)  # noqa: E731
+    else:
+        n = c["n"]
+        qd, kc, vc = W.decode_inputs(1, 32, 8, 128, n, seed=6)
+        qd, kc, vc = qd.to(dev), kc.to(dev), vc.to(dev)
+        ws = torch.empty(jl.decode_workspace_size(1, 32, 8, 128, n - 1), dtype=torch.uint8,
+                         device=dev)
+        fn = lambda: jl.bifocal_decode(qd, kc, vc, n - 1, w_local=2048,  # noqa: E731
+                                       w_pretrained=32768, rope_base=1e6, workspace=ws)
+    for _ in range(args.warmup + args.steps):
+        fn()
+    jl.check_device_status()
+    print(json.dumps({"case": args.case, "launch_groups": args.warmup + args.steps}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=sorted(CASES), default=None,
+                    help="run one small profiling case instead of the benchmark")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "cuda":
+        args.warmup = 3
+    if args.case:
+        run_case(args)
+    elif args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

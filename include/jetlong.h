@@ -1,0 +1,157 @@
+/*
+ * jetlong.h -- C ABI of libjetlong: dynamic bifocal RoPE attention on B200
+ * (sm_100a).
+ *
+ * The method (Jet-Long, "Efficient long-context extension with dynamic bifocal
+ * RoPE"):
+ *   - G = max(1, ceil(L / w_pretrained)) is recomputed from the current length L
+ *     (bittide paper summary §3.1, group-size equation; techwalker explainer §二).
+ *   - f(x) = floor(x / G) maps remote positions back onto the pretrained grid
+ *     (bittide summary §3.1, position-map equation).
+ *   - A causal pair (query q, key k <= q) with q - k < w_local is LOCAL and uses
+ *     standard RoPE at (q, k); every other pair is REMOTE and uses RoPE at
+ *     (f(q), f(k)) (techwalker §二, bittide §3.2).  G = 1 is exactly plain
+ *     causal RoPE attention.
+ *   - Prefill merges the two windows with LogSumExp weights (techwalker §四,
+ *     bittide §3.2); decode keeps the cache at original positions and applies the
+ *     corrections dq = f(q) - q and dk = f(k) - k in registers (techwalker §三,
+ *     bittide §3.3).
+ *
+ * Conventions for every entry point
+ *   - RoPE pairs are rotate-half: (x_i, x_{i+D/2}) rotated by pos * theta_i with
+ *     theta_i = rope_base^(-2i/D).  q and k passed to prefill are PRE-RoPE.
+ *   - Softmax scale defaults to 1/sqrt(D).  lse is the natural log of
+ *     sum_k exp(scale * score_k), in fp32.
+ *   - All tensor pointers are caller-owned DEVICE memory, contiguous, 16-byte
+ *     aligned.  The library writes only `out`, `lse` and the workspace.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  No entry point synchronises the host with the device except the
+ *     first call that builds or grows a library-owned table (see below) and
+ *     jl_check_device_status.
+ *   - Arguments are validated before anything is launched.  A rejected call
+ *     returns JL_ERR_INVALID_ARG or JL_ERR_UNSUPPORTED, launches nothing and
+ *     leaves a message for jl_last_error().  No C++ exception crosses the ABI
+ *     and no kernel traps.
+ *   - Library-owned device memory: per device, a cos/sin table of the RoPE
+ *     angles (fp64 sincos rounded to fp32, [positions][D/2] pairs) grown on
+ *     demand, a 4-byte device status word, and, for jl_bifocal_prefill only, a
+ *     grown scratch buffer.  jl_finalize releases them.  The first call that
+ *     creates or grows them allocates and synchronises, so make it before any
+ *     stream capture.
+ */
+#ifndef JETLONG_H
+#define JETLONG_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st *jl_stream_t;
+
+typedef enum {
+  JL_OK = 0,
+  JL_ERR_INVALID_ARG = 1, /* a null/misaligned pointer, a bad size or shape */
+  JL_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. head dim) */
+  JL_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed */
+  JL_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired (device status) */
+} jl_status;
+
+typedef enum { JL_BF16 = 0, JL_F32 = 1 } jl_dtype;
+
+enum {
+  /* Run the same kernels with the bifocal rule switched off: every pair takes
+   * standard RoPE at its original positions (plain causal RoPE attention).
+   * This is the overhead baseline; with G = 1 the bifocal call takes exactly
+   * this path. */
+  JL_FLAG_NO_BIFOCAL = 1u << 0
+};
+
+/* G = max(1, ceil(L / w_pretrained)) (bittide summary §3.1).  Returns -1 when
+ * L < 1 or w_pretrained < 1.  Host-only. */
+long long jl_group_size(long long L, long long w_pretrained);
+
+/*
+ * Bifocal prefill, bf16 (techwalker §四; bittide §3.2, §3.4).
+ *   q    [B, L, Hq, D]  bf16, pre-RoPE, query at position l is row l
+ *   k, v [B, L, Hkv, D] bf16, k pre-RoPE; Hq % Hkv == 0 (grouped-query heads:
+ *                       query head h reads kv head h / (Hq / Hkv))
+ *   out  [B, L, Hq, D]  bf16 (written)
+ *   lse  [B, Hq, L]     fp32 (written)
+ *   D == 128.  w_local >= 0 (0 = every pair remote), w_pretrained >= 1,
+ *   rope_base > 1.  The library's scratch buffer holds the rotated keys
+ *   (2 * B * L * Hkv * D bf16); it is grown on demand.
+ */
+jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v,
+                             void *out, float *lse, int B, int L, int Hq,
+                             int Hkv, int D, int w_local, int w_pretrained,
+                             double rope_base, jl_stream_t stream);
+
+/* Bytes of caller workspace jl_bifocal_prefill_ex needs (0 for fp32). */
+size_t jl_bifocal_prefill_workspace_size(int B, int L, int Hkv, int D,
+                                         jl_dtype dtype);
+
+/*
+ * Bifocal prefill with every option.  dtype JL_BF16 (D == 128, tensor cores)
+ * or JL_F32 (D in {64, 128}, fp32 CUDA-core kernel; out is fp32).
+ * softmax_scale <= 0 selects 1/sqrt(D).  flags: JL_FLAG_NO_BIFOCAL.
+ * workspace: device memory of at least jl_bifocal_prefill_workspace_size()
+ * bytes, 256-byte aligned; NULL selects the library-owned buffer.
+ */
+jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v,
+                                void *out, float *lse, int B, int L, int Hq,
+                                int Hkv, int D, int w_local, int w_pretrained,
+                                double rope_base, jl_dtype dtype,
+                                float softmax_scale, unsigned flags,
+                                void *workspace, size_t workspace_bytes,
+                                jl_stream_t stream);
+
+/* Bytes of workspace jl_bifocal_decode needs for these sizes. */
+size_t jl_bifocal_decode_workspace_size(int B, int Hq, int Hkv, int D, int pos);
+
+/*
+ * Single-token bifocal decode, bf16 (techwalker §三; bittide §3.3).
+ *   q_new          [B, Hq, D] bf16, pre-RoPE, the token at position `pos`
+ *   k_cache_roped  [B, cache_capacity, Hkv, D] bf16, keys already rotated by
+ *                  standard RoPE at their original positions; slots 0..pos are
+ *                  valid and slot pos holds the new token's key
+ *   v_cache        [B, cache_capacity, Hkv, D] bf16
+ *   out [B, Hq, D] bf16 and lse [B, Hq] fp32 (written)
+ *   G is computed from L = pos + 1.  Keys with pos - k < w_local take no
+ *   correction; farther keys are rotated by dk = f(k) - k in registers, and the
+ *   query by dq = f(pos) - pos.  The caches are never written.
+ *   workspace: device memory of at least jl_bifocal_decode_workspace_size()
+ *   bytes, 16-byte aligned (split-KV partial results).
+ *   D == 128, 0 <= pos < cache_capacity, Hq % Hkv == 0.
+ *   flags: JL_FLAG_NO_BIFOCAL.
+ */
+jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped,
+                            const void *v_cache, int pos, int cache_capacity,
+                            void *out, float *lse, void *workspace,
+                            size_t workspace_bytes, int B, int Hq, int Hkv,
+                            int D, int w_local, int w_pretrained,
+                            double rope_base, unsigned flags,
+                            jl_stream_t stream);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char *jl_last_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status
+ * word.  Returns JL_ERR_TIMEOUT if a kernel gave up a bounded wait since the
+ * last check (its outputs are then invalid), JL_ERR_CUDA on a CUDA error,
+ * JL_OK otherwise.
+ */
+jl_status jl_check_device_status(jl_stream_t stream);
+
+/* Releases every library-owned device buffer on every device (synchronises
+ * each device first).  Later calls re-create them. */
+void jl_finalize(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JETLONG_H */

@@ -1,0 +1,188 @@
+"""Dynamic bifocal RoPE attention (Jet-Long) on B200 -- Python binding.
+
+Thin ctypes layer over ``libjetlong.so`` (C ABI declared in include/jetlong.h):
+it checks tensor dtypes/devices/shapes, passes raw device pointers, sizes and
+the current CUDA stream, and turns a non-OK status into an exception.  Every
+step of the computation runs in the library's sm_100a kernels; there is no
+fallback.  If the shared library is missing, the first call raises.
+
+PyTorch is used only for device memory and streams.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "NO_BIFOCAL", "JetLongError", "group_size", "bifocal_prefill",
+    "prefill_workspace_size", "decode_workspace_size", "bifocal_decode",
+    "check_device_status", "finalize", "library_path", "load",
+]
+
+NO_BIFOCAL = 1 << 0  # JL_FLAG_NO_BIFOCAL
+
+_BF16, _F32 = 0, 1
+_STATUS = {0: "JL_OK", 1: "JL_ERR_INVALID_ARG", 2: "JL_ERR_UNSUPPORTED",
+           3: "JL_ERR_CUDA", 4: "JL_ERR_TIMEOUT"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lib = None
+
+
+class JetLongError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def library_path() -> str:
+    return os.environ.get("JETLONG_LIB", os.path.join(_HERE, "libjetlong.so"))
+
+
+def load():
+    """Load libjetlong.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise ImportError(
+            f"libjetlong.so not found at {path}; build it with "
+            "`python -m long_context_attention_bifocal_b200.build` (there is no fallback)")
+    L = ctypes.CDLL(path)
+    p, i, d, u, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_uint,
+                      ctypes.c_size_t)
+    L.jl_group_size.restype = ctypes.c_longlong
+    L.jl_group_size.argtypes = [ctypes.c_longlong, ctypes.c_longlong]
+    L.jl_bifocal_prefill.restype = i
+    L.jl_bifocal_prefill.argtypes = [p, p, p, p, p, i, i, i, i, i, i, i, d, p]
+    L.jl_bifocal_prefill_workspace_size.restype = sz
+    L.jl_bifocal_prefill_workspace_size.argtypes = [i, i, i, i, i]
+    L.jl_bifocal_prefill_ex.restype = i
+    L.jl_bifocal_prefill_ex.argtypes = [p, p, p, p, p, i, i, i, i, i, i, i, d, i,
+                                        ctypes.c_float, u, p, sz, p]
+    L.jl_bifocal_decode_workspace_size.restype = sz
+    L.jl_bifocal_decode_workspace_size.argtypes = [i, i, i, i, i]
+    L.jl_bifocal_decode.restype = i
+    L.jl_bifocal_decode.argtypes = [p, p, p, i, i, p, p, p, sz, i, i, i, i, i, i, d,
+                                    u, p]
+    L.jl_last_error.restype = ctypes.c_char_p
+    L.jl_last_error.argtypes = []
+    L.jl_check_device_status.restype = i
+    L.jl_check_device_status.argtypes = [p]
+    L.jl_finalize.restype = None
+    L.jl_finalize.argtypes = []
+    _lib = L
+    return L
+
+
+def _check(status):
+    if status != 0:
+        msg = load().jl_last_error().decode(errors="replace")
+        raise JetLongError(status, msg)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def group_size(L: int, w_pretrained: int) -> int:
+    """G = max(1, ceil(L / w_pretrained)) as the library computes it."""
+    return int(load().jl_group_size(L, w_pretrained))
+
+
+def prefill_workspace_size(B, L, Hkv, D, dtype=torch.bfloat16) -> int:
+    code = _BF16 if dtype == torch.bfloat16 else _F32
+    return int(load().jl_bifocal_prefill_workspace_size(B, L, Hkv, D, code))
+
+
+def bifocal_prefill(q, k, v, *, w_local, w_pretrained, rope_base, out=None, lse=None,
+                    softmax_scale=0.0, flags=0, workspace=None, stream=None):
+    """Bifocal causal prefill.  q [B,L,Hq,D], k/v [B,L,Hkv,D] (pre-RoPE),
+    bf16 (D=128) or fp32 (D in {64,128}).  Returns (out [B,L,Hq,D], lse [B,Hq,L] fp32).
+    """
+    dtype = q.dtype
+    if dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("q must be bfloat16 or float32")
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _need(q, "q", dtype)
+    _need(k, "k", dtype, (B, L, Hkv, D))
+    _need(v, "v", dtype, (B, L, Hkv, D))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    _need(out, "out", dtype, (B, L, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq, L))
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8)
+        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel()
+    with torch.cuda.device(q.device):
+        _check(load().jl_bifocal_prefill_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, L, Hq, Hkv, D,
+            int(w_local), int(w_pretrained), float(rope_base),
+            _BF16 if dtype == torch.bfloat16 else _F32, float(softmax_scale),
+            int(flags), ws_ptr, ws_bytes, _stream(stream)))
+    return out, lse
+
+
+def decode_workspace_size(B, Hq, Hkv, D, pos) -> int:
+    return int(load().jl_bifocal_decode_workspace_size(B, Hq, Hkv, D, pos))
+
+
+def bifocal_decode(q_new, k_cache, v_cache, pos, *, w_local, w_pretrained, rope_base,
+                   out=None, lse=None, workspace=None, flags=0, stream=None):
+    """Single-token decode at position `pos`.  q_new [B,Hq,D] pre-RoPE bf16;
+    caches [B,cap,Hkv,D] bf16 with keys rotated at their original positions.
+    Returns (out [B,Hq,D] bf16, lse [B,Hq] fp32)."""
+    B, Hq, D = q_new.shape
+    cap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _need(q_new, "q_new", torch.bfloat16)
+    _need(k_cache, "k_cache", torch.bfloat16, (B, cap, Hkv, D))
+    _need(v_cache, "v_cache", torch.bfloat16, (B, cap, Hkv, D))
+    if out is None:
+        out = torch.empty_like(q_new)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q_new.device)
+    _need(out, "out", torch.bfloat16, (B, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq))
+    if workspace is None:
+        n = decode_workspace_size(B, Hq, Hkv, D, pos)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q_new.device)
+    _need(workspace, "workspace", torch.uint8)
+    with torch.cuda.device(q_new.device):
+        _check(load().jl_bifocal_decode(
+            _ptr(q_new), _ptr(k_cache), _ptr(v_cache), int(pos), cap, _ptr(out),
+            _ptr(lse), _ptr(workspace), workspace.numel(), B, Hq, Hkv, D, int(w_local),
+            int(w_pretrained), float(rope_base), int(flags), _stream(stream)))
+    return out, lse
+
+
+def check_device_status(stream=None):
+    """Synchronise `stream`; raise JetLongError if a kernel abandoned a bounded wait."""
+    _check(load().jl_check_device_status(_stream(stream)))
+
+
+def finalize():
+    load().jl_finalize()

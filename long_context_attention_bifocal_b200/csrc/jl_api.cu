@@ -1,0 +1,402 @@
+// jl_api.cu -- the C ABI of libjetlong: argument validation, the method's
+// scalar parameters, library-owned per-device state, and kernel dispatch.
+//
+// Scalar parameters (Jet-Long, bittide paper summary §3.1; techwalker
+// explainer §二):  G = max(1, ceil(L / w_pretrained)), recomputed from the
+// current length (prefill: the prompt length; decode: pos + 1).  With G = 1
+// the remap f(x) = floor(x/G) is the identity and both windows use the same
+// RoPE, so the call takes exactly the non-bifocal path (every pair "local");
+// the same holds when the local window covers every pair.
+#include <climits>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "jl_internal.h"
+
+namespace jl {
+
+namespace {
+
+thread_local std::string g_last_error;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  std::mutex mu;
+  bool init = false;
+  int sms = 0;
+  float2 *table = nullptr;
+  int table_positions = 0;
+  int table_D = 0;
+  double table_base = 0.0;
+  unsigned *status = nullptr;
+  void *scratch = nullptr;
+  size_t scratch_bytes = 0;
+};
+
+DeviceState g_dev[kMaxDevices];
+
+jl_status current(DeviceState **out, int *dev_out = nullptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(JL_ERR_UNSUPPORTED, "device %d out of range", dev);
+  DeviceState &d = g_dev[dev];
+  std::lock_guard<std::mutex> lock(d.mu);
+  if (!d.init) {
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+    if (prop.major != 10 || prop.minor != 0)
+      return fail(JL_ERR_UNSUPPORTED,
+                  "libjetlong is built for sm_100a (B200); device %d is sm_%d%d", dev,
+                  prop.major, prop.minor);
+    d.sms = prop.multiProcessorCount;
+    e = cudaMalloc(&d.status, 256);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(status)");
+    e = cudaMemset(d.status, 0, 256);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(status)");
+    d.init = true;
+  }
+  *out = &d;
+  if (dev_out) *dev_out = dev;
+  return JL_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+long long group_size_ll(long long L, long long w) {
+  if (L < 1 || w < 1) return -1;
+  const long long g = (L + w - 1) / w;
+  return g < 1 ? 1 : g;
+}
+
+}  // namespace
+
+jl_status fail(jl_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+jl_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(JL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int sm_count() {
+  DeviceState *d = nullptr;
+  if (current(&d) != JL_OK) return 148;
+  return d->sms;
+}
+
+jl_status rope_table(int D, double base, int min_positions, cudaStream_t s, RopeTable *out) {
+  DeviceState *d = nullptr;
+  jl_status st = current(&d);
+  if (st != JL_OK) return st;
+  std::lock_guard<std::mutex> lock(d->mu);
+  if (d->table == nullptr || d->table_D != D || d->table_base != base ||
+      d->table_positions < min_positions) {
+    int want = min_positions < 4096 ? 4096 : min_positions;
+    if (d->table && d->table_D == D && d->table_base == base && want < 2 * d->table_positions)
+      want = 2 * d->table_positions;
+    want = ((want + 4095) / 4096) * 4096;
+    if (d->table) {
+      cudaError_t e = cudaDeviceSynchronize();  // earlier kernels may still read it
+      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+      cudaFree(d->table);
+      d->table = nullptr;
+      d->table_positions = 0;
+    }
+    float2 *t = nullptr;
+    cudaError_t e = cudaMalloc(&t, sizeof(float2) * static_cast<size_t>(want) * (D / 2));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(rope table)");
+    e = launch_rope_table(t, want, D, base, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // usable from any stream after this
+    if (e != cudaSuccess) {
+      cudaFree(t);
+      return cuda_fail(e, "rope table build");
+    }
+    d->table = t;
+    d->table_positions = want;
+    d->table_D = D;
+    d->table_base = base;
+  }
+  out->cs = d->table;
+  out->positions = d->table_positions;
+  out->half = D / 2;
+  return JL_OK;
+}
+
+jl_status status_word(unsigned **out) {
+  DeviceState *d = nullptr;
+  jl_status st = current(&d);
+  if (st != JL_OK) return st;
+  *out = d->status;
+  return JL_OK;
+}
+
+jl_status prefill_scratch(size_t bytes, void **out) {
+  DeviceState *d = nullptr;
+  jl_status st = current(&d);
+  if (st != JL_OK) return st;
+  std::lock_guard<std::mutex> lock(d->mu);
+  if (d->scratch_bytes < bytes) {
+    if (d->scratch) {
+      cudaError_t e = cudaDeviceSynchronize();
+      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+      cudaFree(d->scratch);
+      d->scratch = nullptr;
+      d->scratch_bytes = 0;
+    }
+    void *p = nullptr;
+    cudaError_t e = cudaMalloc(&p, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(prefill scratch)");
+    d->scratch = p;
+    d->scratch_bytes = bytes;
+  }
+  *out = d->scratch;
+  return JL_OK;
+}
+
+}  // namespace jl
+
+using namespace jl;
+
+namespace {
+
+size_t prefill_ws_bytes(int B, int L, int Hkv, int D) {
+  const size_t one = static_cast<size_t>(B) * L * Hkv * D * sizeof(__nv_bfloat16);
+  const size_t aligned = (one + 255) & ~static_cast<size_t>(255);
+  return 2 * aligned;  // rotated keys at original and at remapped positions
+}
+
+jl_status check_common(int B, int L, int Hq, int Hkv, int D, int w_local, int w_pretrained,
+                       double rope_base) {
+  if (B < 1 || L < 1 || Hq < 1 || Hkv < 1)
+    return fail(JL_ERR_INVALID_ARG, "sizes must be >= 1 (B=%d L=%d Hq=%d Hkv=%d)", B, L, Hq, Hkv);
+  if (Hq % Hkv != 0)
+    return fail(JL_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  if (D < 2 || D % 2 != 0) return fail(JL_ERR_INVALID_ARG, "head dim %d must be even", D);
+  if (w_local < 0) return fail(JL_ERR_INVALID_ARG, "w_local must be >= 0 (got %d)", w_local);
+  if (w_pretrained < 1)
+    return fail(JL_ERR_INVALID_ARG, "w_pretrained must be >= 1 (got %d)", w_pretrained);
+  if (!(rope_base > 1.0) || !std::isfinite(rope_base))
+    return fail(JL_ERR_INVALID_ARG, "rope_base must be a finite number > 1");
+  return JL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+long long jl_group_size(long long L, long long w_pretrained) {
+  return group_size_ll(L, w_pretrained);
+}
+
+const char *jl_last_error(void) { return g_last_error.c_str(); }
+
+size_t jl_bifocal_prefill_workspace_size(int B, int L, int Hkv, int D, jl_dtype dtype) {
+  if (B < 1 || L < 1 || Hkv < 1 || D < 1) return 0;
+  if (dtype != JL_BF16) return 0;
+  return prefill_ws_bytes(B, L, Hkv, D);
+}
+
+jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v, void *out,
+                                float *lse, int B, int L, int Hq, int Hkv, int D,
+                                int w_local, int w_pretrained, double rope_base,
+                                jl_dtype dtype, float softmax_scale, unsigned flags,
+                                void *workspace, size_t workspace_bytes,
+                                jl_stream_t stream) {
+  g_last_error.clear();
+  jl_status st = check_common(B, L, Hq, Hkv, D, w_local, w_pretrained, rope_base);
+  if (st != JL_OK) return st;
+  if (!q || !k || !v || !out || !lse)
+    return fail(JL_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(JL_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL)) != 0)
+    return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if (dtype != JL_BF16 && dtype != JL_F32)
+    return fail(JL_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dtype));
+  if (dtype == JL_BF16 && D != 128)
+    return fail(JL_ERR_UNSUPPORTED, "bf16 prefill supports head dim 128 (got %d)", D);
+  if (dtype == JL_F32 && D != 64 && D != 128)
+    return fail(JL_ERR_UNSUPPORTED, "fp32 prefill supports head dim 64 or 128 (got %d)", D);
+  if (static_cast<long long>((L + 127) / 128) * B * Hq >= (1LL << 31))
+    return fail(JL_ERR_UNSUPPORTED, "problem too large for one launch");
+  if (!(softmax_scale >= 0.f) && !(softmax_scale < 0.f))
+    return fail(JL_ERR_INVALID_ARG, "softmax_scale is NaN");
+  const size_t need_ws = dtype == JL_BF16 ? prefill_ws_bytes(B, L, Hkv, D) : 0;
+  if (workspace != nullptr) {
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return fail(JL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (workspace_bytes < need_ws)
+      return fail(JL_ERR_INVALID_ARG, "workspace too small: %zu bytes, need %zu",
+                  workspace_bytes, need_ws);
+  }
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long G = group_size_ll(L, w_pretrained);
+  const bool plain = (flags & JL_FLAG_NO_BIFOCAL) || G == 1 || w_local >= L;
+  PrefillArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.lse = lse;
+  a.B = B;
+  a.L = L;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.D = D;
+  a.G = static_cast<int>(G);
+  a.w_eff = plain ? INT_MAX : w_local;
+  a.scale = softmax_scale > 0.f ? softmax_scale : static_cast<float>(1.0 / std::sqrt(D));
+  a.kstd = a.krem = nullptr;
+  st = rope_table(D, rope_base, L, s, &a.table);
+  if (st != JL_OK) return st;
+  st = status_word(&a.status);
+  if (st != JL_OK) return st;
+
+  if (dtype == JL_F32) {
+    cudaError_t e = launch_prefill_f32(a, s);
+    return e == cudaSuccess ? JL_OK : cuda_fail(e, "fp32 prefill launch");
+  }
+
+  void *ws = workspace;
+  if (ws == nullptr) {
+    st = prefill_scratch(need_ws, &ws);
+    if (st != JL_OK) return st;
+  }
+  const size_t one = need_ws / 2;
+  __nv_bfloat16 *kstd = static_cast<__nv_bfloat16 *>(ws);
+  __nv_bfloat16 *krem =
+      reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + one);
+  const bool need_std = a.w_eff > 0;
+  const bool need_rem = !plain;  // some pair is remote
+  cudaError_t e = launch_rotate_keys(static_cast<const __nv_bfloat16 *>(k),
+                                     need_std ? kstd : nullptr, need_rem ? krem : nullptr,
+                                     a.table, B, L, Hkv, D, a.G, s);
+  if (e != cudaSuccess) return cuda_fail(e, "key rotation launch");
+  a.kstd = need_std ? kstd : nullptr;
+  a.krem = need_rem ? krem : nullptr;
+  e = launch_prefill_sm100(a, s);
+  return e == cudaSuccess ? JL_OK : cuda_fail(e, "prefill launch");
+}
+
+jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v, void *out,
+                             float *lse, int B, int L, int Hq, int Hkv, int D, int w_local,
+                             int w_pretrained, double rope_base, jl_stream_t stream) {
+  return jl_bifocal_prefill_ex(q, k, v, out, lse, B, L, Hq, Hkv, D, w_local, w_pretrained,
+                               rope_base, JL_BF16, 0.f, 0u, nullptr, 0, stream);
+}
+
+size_t jl_bifocal_decode_workspace_size(int B, int Hq, int Hkv, int D, int pos) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || pos < 0 || Hq % Hkv != 0) return 0;
+  // the remote/local split adds at most one chunk
+  int chunk = 0, n_far = 0, n_chunks = 0;
+  decode_plan(B, Hq, Hkv, pos, 0, &chunk, &n_far, &n_chunks);
+  return decode_ws_floats(B, Hq, D, n_chunks + 1) * sizeof(float);
+}
+
+jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped, const void *v_cache,
+                            int pos, int cache_capacity, void *out, float *lse,
+                            void *workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                            int D, int w_local, int w_pretrained, double rope_base,
+                            unsigned flags, jl_stream_t stream) {
+  g_last_error.clear();
+  jl_status st = check_common(B, 1, Hq, Hkv, D, w_local, w_pretrained, rope_base);
+  if (st != JL_OK) return st;
+  if (!q_new || !k_cache_roped || !v_cache || !out || !lse || !workspace)
+    return fail(JL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q_new) || !aligned16(k_cache_roped) || !aligned16(v_cache) ||
+      !aligned16(out) || !aligned16(lse) || !aligned16(workspace))
+    return fail(JL_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL)) != 0)
+    return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if (D != 128) return fail(JL_ERR_UNSUPPORTED, "decode supports head dim 128 (got %d)", D);
+  if (cache_capacity < 1 || pos < 0 || pos >= cache_capacity)
+    return fail(JL_ERR_INVALID_ARG, "need 0 <= pos (%d) < cache_capacity (%d)", pos,
+                cache_capacity);
+  const size_t need = jl_bifocal_decode_workspace_size(B, Hq, Hkv, D, pos);
+  if (workspace_bytes < need)
+    return fail(JL_ERR_INVALID_ARG, "workspace too small: %zu bytes, need %zu",
+                workspace_bytes, need);
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long G = group_size_ll(static_cast<long long>(pos) + 1, w_pretrained);
+  const bool plain = (flags & JL_FLAG_NO_BIFOCAL) || G == 1;
+  DecodeArgs a;
+  a.q = static_cast<const __nv_bfloat16 *>(q_new);
+  a.kc = static_cast<const __nv_bfloat16 *>(k_cache_roped);
+  a.vc = static_cast<const __nv_bfloat16 *>(v_cache);
+  a.out = static_cast<__nv_bfloat16 *>(out);
+  a.lse = lse;
+  a.ws = static_cast<float *>(workspace);
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.D = D;
+  a.pos = pos;
+  a.cap = cache_capacity;
+  a.G = static_cast<int>(G);
+  // keys k <= pos - w_local are remote
+  const long long fe = static_cast<long long>(pos) + 1 - w_local;
+  a.far_end = plain ? 0 : static_cast<int>(fe < 0 ? 0 : fe);
+  a.scale = static_cast<float>(1.0 / std::sqrt(D));
+  decode_plan(B, Hq, Hkv, pos, a.far_end, &a.chunk, &a.n_far_chunks, &a.n_chunks);
+  st = rope_table(D, rope_base, pos + 1 < 64 ? 64 : pos + 1, s, &a.table);
+  if (st != JL_OK) return st;
+  cudaError_t e = launch_decode(a, s);
+  return e == cudaSuccess ? JL_OK : cuda_fail(e, "decode launch");
+}
+
+jl_status jl_check_device_status(jl_stream_t stream) {
+  g_last_error.clear();
+  DeviceState *d = nullptr;
+  jl_status st = current(&d);
+  if (st != JL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned word = 0;
+  e = cudaMemcpy(&word, d->status, sizeof word, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  if (word != 0) {
+    cudaMemset(d->status, 0, sizeof word);
+    return fail(JL_ERR_TIMEOUT, "a kernel abandoned a bounded wait (status 0x%x)", word);
+  }
+  return JL_OK;
+}
+
+void jl_finalize(void) {
+  int prev = 0;
+  const bool have_prev = cudaGetDevice(&prev) == cudaSuccess;
+  for (int i = 0; i < kMaxDevices; ++i) {
+    DeviceState &d = g_dev[i];
+    std::lock_guard<std::mutex> lock(d.mu);
+    if (!d.init) continue;
+    if (cudaSetDevice(i) != cudaSuccess) continue;
+    cudaDeviceSynchronize();
+    if (d.table) cudaFree(d.table);
+    if (d.status) cudaFree(d.status);
+    if (d.scratch) cudaFree(d.scratch);
+    d.table = nullptr;
+    d.status = nullptr;
+    d.scratch = nullptr;
+    d.table_positions = 0;
+    d.scratch_bytes = 0;
+    d.init = false;
+  }
+  if (have_prev) cudaSetDevice(prev);
+}
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+// jl_internal.h -- declarations shared by the translation units of libjetlong.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "jetlong.h"
+
+namespace jl {
+
+// Status-word bits written by kernels (never a trap).
+enum : unsigned {
+  kStatusTimeout = 1u << 0,  // a bounded mbarrier wait expired
+  kStatusBounds = 1u << 1,   // an index check refused an access
+};
+
+// Angle table: cs[p * half + i] = (cos(p * theta_i), sin(p * theta_i)),
+// computed with fp64 sincos and rounded to fp32.
+struct RopeTable {
+  const float2 *cs;
+  int positions;  // valid p in [0, positions)
+  int half;       // D / 2
+};
+
+// Records a message for jl_last_error() and returns st.
+jl_status fail(jl_status st, const char *fmt, ...);
+jl_status cuda_fail(cudaError_t e, const char *what);
+
+// Per-device library state (current device).
+jl_status rope_table(int D, double base, int min_positions, cudaStream_t s,
+                     RopeTable *out);
+jl_status status_word(unsigned **out);
+jl_status prefill_scratch(size_t bytes, void **out);
+int sm_count();
+
+// ---- launchers (each returns the launch's cudaError_t) ----
+cudaError_t launch_rope_table(float2 *cs, int positions, int D, double base,
+                              cudaStream_t s);
+
+// Rotated copies of the keys of a [B,L,Hkv,D] bf16 tensor:
+// kstd = R(l) k (if kstd), krem = R(floor(l/G)) k (if krem).
+cudaError_t launch_rotate_keys(const __nv_bfloat16 *k, __nv_bfloat16 *kstd,
+                               __nv_bfloat16 *krem, RopeTable t, int B, int L,
+                               int Hkv, int D, int G, cudaStream_t s);
+
+struct PrefillArgs {
+  const void *q;      // [B,L,Hq,D] pre-RoPE
+  const void *kstd;   // [B,L,Hkv,D] keys rotated at original positions (bf16 path)
+  const void *krem;   // [B,L,Hkv,D] keys rotated at floor(l/G)         (bf16 path)
+  const void *k;      // raw keys (fp32 path)
+  const void *v;      // [B,L,Hkv,D]
+  void *out;          // [B,L,Hq,D]
+  float *lse;         // [B,Hq,L]
+  int B, L, Hq, Hkv, D;
+  int G;
+  int w_eff;          // local iff q - k < w_eff (INT_MAX: every pair local)
+  float scale;        // softmax scale
+  RopeTable table;
+  unsigned *status;
+};
+
+cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s);
+cudaError_t launch_prefill_f32(const PrefillArgs &a, cudaStream_t s);
+
+struct DecodeArgs {
+  const __nv_bfloat16 *q;   // [B,Hq,D] pre-RoPE
+  const __nv_bfloat16 *kc;  // [B,cap,Hkv,D] rotated at original positions
+  const __nv_bfloat16 *vc;  // [B,cap,Hkv,D]
+  __nv_bfloat16 *out;       // [B,Hq,D]
+  float *lse;               // [B,Hq]
+  float *ws;                // split partials
+  int B, Hq, Hkv, D, pos, cap;
+  int G;
+  int far_end;              // keys [0, far_end) take the dk correction
+  float scale;
+  RopeTable table;
+  int chunk;                // keys per split
+  int n_far_chunks, n_chunks;
+};
+
+// Workspace floats for the given split layout.
+size_t decode_ws_floats(int B, int Hq, int D, int n_chunks);
+void decode_plan(int B, int Hq, int Hkv, int pos, int far_end, int *chunk,
+                 int *n_far_chunks, int *n_chunks);
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+
+}  // namespace jl

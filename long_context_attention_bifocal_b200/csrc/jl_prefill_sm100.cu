@@ -1,0 +1,575 @@
+// jl_prefill_sm100.cu -- bifocal prefill attention on the sm_100a tensor cores.
+//
+// What it computes (Jet-Long; techwalker explainer §二/§四, bittide paper
+// summary §3.1-§3.2): causal attention in which a pair (q, k) with
+// q - k < w_local scores <R(q)Q, R(k)K> and every farther pair scores
+// <R(f(q))Q, R(f(k))K>, f(x) = floor(x/G).  The pages reach this with three
+// flash-attention calls merged by LogSumExp weights (B: full causal at
+// remapped positions, A: local band at original positions, C: local band at
+// remapped positions; final = B - C + A).  Here the merge is done per tile
+// instead, with complementary masks, so no subtraction (and no cancellation)
+// happens:
+//   * a kv tile whose pairs are all remote is one pass with remapped RoPE;
+//   * a kv tile whose pairs are all local is one pass with standard RoPE;
+//   * a tile straddling the window edge is two passes over the same keys, one
+//     per class under complementary masks.
+// All passes feed one online softmax (fp32 running max and sum, base 2), so the
+// epilogue's O = acc / l and lse = m + ln l are exactly the LogSumExp-weighted
+// combination of the per-class partial sums.
+//
+// B200 design: one CTA per (batch, query head, 128-row query tile), heaviest
+// tiles first.  Warp roles:
+//   warps 0-3  rotate the Q tile twice (standard and remapped) into swizzled
+//              shared memory, then run the online softmax: thread r owns query
+//              row r = TMEM lane r, reads S from TMEM, writes P (bf16) to shared
+//              memory, rescales O in TMEM when the running max grows by more
+//              than 2^8 (lazy rescale), and finally normalises O and stores it.
+//   warp 4     TMA producer: K tile (pre-rotated copy of the needed class) and
+//              V tile per pass into a 2-stage ring.
+//   warp 5     allocates TMEM and issues every tcgen05.mma from one thread:
+//              S = Q K^T (M=N=128, K=128: 8 x K16 steps) into one of two TMEM
+//              S buffers, and O += P V into the TMEM O accumulator.
+// Every mbarrier wait is bounded (1 s); a thread that gives up raises the
+// CTA's abort flag and the device status word, after which all CTAs drain and
+// return without touching their outputs further.
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <mutex>
+
+#include "jl_internal.h"
+#include "jl_sm100.cuh"
+
+namespace jl {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per tile
+constexpr int kHD = 128;  // head dim
+constexpr int kStages = 2;
+constexpr int kThreads = 192;
+constexpr uint32_t kTileBytes = kBM * kHD * 2;  // one 128x128 bf16 tile
+constexpr uint32_t kHalfBytes = kTileBytes / 2;  // 64 columns (128 B rows)
+
+constexpr uint32_t kOffQs = 0;
+constexpr uint32_t kOffQr = kOffQs + kTileBytes;
+constexpr uint32_t kOffK = kOffQr + kTileBytes;
+constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
+constexpr uint32_t kOffP = kOffV + kStages * kTileBytes;
+constexpr uint32_t kOffBar = kOffP + kTileBytes;
+
+enum : int {
+  kBarQFull = 0,
+  kBarKFull = 1,
+  kBarKEmpty = kBarKFull + kStages,
+  kBarVFull = kBarKEmpty + kStages,
+  kBarVEmpty = kBarVFull + kStages,
+  kBarSFull = kBarVEmpty + kStages,
+  kBarSFree = kBarSFull + 2,
+  kBarPFull = kBarSFree + 2,
+  kBarODone = kBarPFull + 1,
+  kBarDrain = kBarODone + 1,
+  kNumBars = kBarDrain + 1
+};
+
+constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
+constexpr uint32_t kOffSkip = kOffAbort + 4;
+constexpr uint32_t kSmemUsed = kOffSkip + 4;
+constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // room to align the base to 1 KiB
+static_assert(kSmemAlloc <= 232448, "shared memory budget");
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmS0 = 0, kTmS1 = 128, kTmO = 256;
+constexpr uint64_t kTimeoutNs = 1000000000ull;
+
+enum : int { kStd = 0, kRem = 1 };
+enum : int { kMaskNone = 0, kMaskFarOnly = 1, kMaskLocalOnly = 2 };
+
+// The pass sequence of query tile i: for every kv tile j <= i, a remote pass
+// if the tile holds a remote pair, then a local pass if it holds a local pair.
+struct PassIter {
+  int i, w;        // query tile, local window (INT_MAX: every pair local)
+  int j, sub;      // current kv tile, 0/1 = first/second pass of the tile
+  bool two, far0;  // tile holds both classes; first pass is remote
+
+  __device__ bool has_far(int jj) const {
+    return static_cast<long long>(kBN) * (i - jj) + (kBN - 1) >= w;
+  }
+  __device__ bool has_local(int jj) const {
+    long long lo = static_cast<long long>(kBN) * (i - jj) - (kBM - 1);
+    if (lo < 0) lo = 0;
+    return lo < w;
+  }
+  __device__ void load() {
+    const bool f = has_far(j), l = has_local(j);
+    two = f && l;
+    far0 = f;
+  }
+  __device__ void begin(int qi, int wl) {
+    i = qi;
+    w = wl;
+    j = 0;
+    sub = 0;
+    load();
+  }
+  __device__ bool done() const { return j > i; }
+  __device__ int kind() const { return (sub == 0 && far0) ? kRem : kStd; }
+  __device__ int mask() const {
+    return two ? (sub == 0 ? kMaskFarOnly : kMaskLocalOnly) : kMaskNone;
+  }
+  __device__ void next() {
+    if (two && sub == 0) {
+      sub = 1;
+    } else {
+      ++j;
+      sub = 0;
+      if (j <= i) load();
+    }
+  }
+};
+
+struct KParams {
+  const __nv_bfloat16 *q;
+  __nv_bfloat16 *out;
+  float *lse;
+  const float2 *cs;
+  unsigned *status;
+  int B, L, Hq, Hkv, G, w, n_qtiles;
+  float scale_log2;  // softmax scale * log2(e)
+};
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ void raise_abort(volatile int *abort_s, unsigned *status) {
+  *abort_s = 1;
+  atomicOr(status, kStatusTimeout);
+}
+
+// Wait used while draining: only the time limit ends it.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kTimeoutNs) break;
+  }
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8]) {
+  const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    x[2 * j] = __uint_as_float(w4[j] << 16);
+    x[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bifocal_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_kstd,
+                                 const __grid_constant__ CUtensorMap tm_krem,
+                                 const __grid_constant__ CUtensorMap tm_v,
+                                 const KParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int bh = p.B * p.Hq;
+  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x / bh);
+  const int rem = static_cast<int>(blockIdx.x % bh);
+  const int hq = rem % p.Hq;
+  const int b = rem / p.Hq;
+  const int hk = hq / (p.Hq / p.Hkv);
+
+  volatile int *abort_s = reinterpret_cast<volatile int *>(smem + kOffAbort);
+  volatile unsigned *abort_g = p.status;
+  auto bar = [&](int i) { return sb + kOffBar + 8u * static_cast<uint32_t>(i); };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBarQFull), 128);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarSFull + s), 1);
+      mbar_init(bar(kBarSFree + s), 128);
+    }
+    mbar_init(bar(kBarPFull), 128);
+    mbar_init(bar(kBarODone), 1);
+    mbar_init(bar(kBarDrain), 1);
+    *abort_s = 0;
+    *reinterpret_cast<volatile int *>(smem + kOffSkip) = (*abort_g != 0u) ? 1 : 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(sb + kOffTmemSlot, kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + kOffTmemSlot);
+  const bool skip = *reinterpret_cast<volatile int *>(smem + kOffSkip) != 0;
+
+  if (!skip) {
+    if (warp < 4) {
+      // ------------------------------------------------ softmax warpgroup --
+      const int r = threadIdx.x;  // query row within the tile == TMEM lane
+      const int qpos = kBM * qt + r;
+      const bool row_ok = qpos < p.L;
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+      const bool need_rem = p.w != INT_MAX;
+
+      // Q_std = R(q) Q and Q_rem = R(f(q)) Q, bf16, in the swizzled K-major
+      // layout the UMMA descriptors expect (two 64-column halves).
+      {
+        const int pr = qpos / p.G;
+        const __nv_bfloat16 *qrow =
+            p.q + ((static_cast<int64_t>(b) * p.L + (row_ok ? qpos : 0)) * p.Hq + hq) * kHD;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          float x1[8], x2[8];
+          if (row_ok) {
+            unpack8(*reinterpret_cast<const uint4 *>(qrow + 8 * c), x1);
+            unpack8(*reinterpret_cast<const uint4 *>(qrow + 64 + 8 * c), x2);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x1[e] = x2[e] = 0.f;
+          }
+#pragma unroll
+          for (int pass = 0; pass < 2; ++pass) {
+            if (pass == 1 && !need_rem) break;
+            const int pos = row_ok ? (pass == 0 ? qpos : pr) : 0;
+            const float2 *t = p.cs + static_cast<int64_t>(pos) * 64 + 8 * c;
+            uint32_t lo[4], hi[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 r0 = __ldg(t + 2 * e), r1 = __ldg(t + 2 * e + 1);
+              lo[e] = pack_bf16x2(x1[2 * e] * r0.x - x2[2 * e] * r0.y,
+                                  x1[2 * e + 1] * r1.x - x2[2 * e + 1] * r1.y);
+              hi[e] = pack_bf16x2(x1[2 * e] * r0.y + x2[2 * e] * r0.x,
+                                  x1[2 * e + 1] * r1.y + x2[2 * e + 1] * r1.x);
+            }
+            uint8_t *dst = smem + (pass == 0 ? kOffQs : kOffQr);
+            *reinterpret_cast<uint4 *>(dst + swz(r, c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            *reinterpret_cast<uint4 *>(dst + kHalfBytes + swz(r, c)) =
+                make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(kBarQFull));
+
+      float m = -INFINITY, l = 0.f;
+      PassIter t;
+      t.begin(qt, p.w);
+      int it = 0;
+      bool ok = true;
+      while (!t.done()) {
+        const int sbuf = it & 1;
+        const uint32_t sph = (it >> 1) & 1;
+        if (!mbar_wait(bar(kBarSFull + sbuf), sph, abort_s, abort_g, kTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float s[128];
+        {
+          const uint32_t col = lane_base + (sbuf ? kTmS1 : kTmS0);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(col + 32 * c, s + 32 * c);
+        }
+        tc_fence_before();
+        mbar_arrive(bar(kBarSFree + sbuf));
+
+        // scores in log2 units; masked entries -> -inf
+        const int k0 = kBN * t.j;
+        const int mk = t.mask();
+        const bool causal = (t.j == qt);
+        float mt = -INFINITY;
+        if (!causal && mk == kMaskNone) {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) {
+            s[e] *= p.scale_log2;
+            mt = fmaxf(mt, s[e]);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) {
+            const int dd = qpos - (k0 + e);
+            bool valid = !causal || dd >= 0;
+            if (mk == kMaskFarOnly) valid = valid && dd >= p.w;
+            if (mk == kMaskLocalOnly) valid = valid && dd < p.w;
+            s[e] = valid ? s[e] * p.scale_log2 : -INFINITY;
+            mt = fmaxf(mt, s[e]);
+          }
+        }
+        const float m_new = fmaxf(m, mt);
+        float alpha = 1.f;
+        bool resc = false;
+        if (m_new > m + 8.f) {  // lazy rescale: only when the max grows by > 2^8
+          alpha = ex2_approx(m - m_new);
+          m = m_new;
+          resc = true;
+        }
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        float rs = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          const float p0 = ex2_approx(s[2 * e] - mu);
+          const float p1 = ex2_approx(s[2 * e + 1] - mu);
+          rs += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        if (it > 0) {
+          // PV of the previous pass done: P buffer free, O stable
+          if (!mbar_wait(bar(kBarODone), (it - 1) & 1, abort_s, abort_g, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (resc && l > 0.f) {
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              float o[32];
+              tmem_ld32(lane_base + kTmO + 32 * c, o);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] *= alpha;
+              tmem_st32(lane_base + kTmO + 32 * c, o);
+            }
+          }
+        }
+        l = l * alpha + rs;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          uint8_t *dst = smem + kOffP + (c >> 3) * kHalfBytes + swz(r, c & 7);
+          *reinterpret_cast<uint4 *>(dst) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPFull));
+        t.next();
+        ++it;
+      }
+      if (ok && !mbar_wait(bar(kBarODone), (it - 1) & 1, abort_s, abort_g, kTimeoutNs))
+        ok = false;
+      if (!ok) {
+        raise_abort(abort_s, p.status);
+      } else {
+        tc_fence_after();
+        const float inv = 1.f / l;
+        __nv_bfloat16 *orow =
+            p.out + ((static_cast<int64_t>(b) * p.L + (row_ok ? qpos : 0)) * p.Hq + hq) * kHD;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32(lane_base + kTmO + 32 * c, o);
+          if (row_ok) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              uint4 w4;
+              w4.x = pack_bf16x2(o[8 * g + 0] * inv, o[8 * g + 1] * inv);
+              w4.y = pack_bf16x2(o[8 * g + 2] * inv, o[8 * g + 3] * inv);
+              w4.z = pack_bf16x2(o[8 * g + 4] * inv, o[8 * g + 5] * inv);
+              w4.w = pack_bf16x2(o[8 * g + 6] * inv, o[8 * g + 7] * inv);
+              *reinterpret_cast<uint4 *>(orow + 32 * c + 8 * g) = w4;
+            }
+          }
+        }
+        if (row_ok)
+          p.lse[(static_cast<int64_t>(b) * p.Hq + hq) * p.L + qpos] =
+              (m + __log2f(l)) * 0.69314718055994530942f;
+      }
+    } else if (warp == 4) {
+      // ------------------------------------------------------ TMA producer --
+      if (lane == 0) {
+        prefetch_tmap(&tm_kstd);
+        prefetch_tmap(&tm_krem);
+        prefetch_tmap(&tm_v);
+        PassIter t;
+        t.begin(qt, p.w);
+        int kiss = 0, viss = 0;  // loads issued
+        while (!t.done()) {
+          const int s = kiss % kStages;
+          const uint32_t ph = (kiss / kStages) & 1;
+          if (!mbar_wait(bar(kBarKEmpty + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
+            raise_abort(abort_s, p.status);
+            break;
+          }
+          const CUtensorMap *km = t.kind() == kStd ? &tm_kstd : &tm_krem;
+          mbar_arrive_expect_tx(bar(kBarKFull + s), kTileBytes);
+          tma_load_4d(sb + kOffK + s * kTileBytes, km, bar(kBarKFull + s), 0, hk, kBN * t.j, b);
+          tma_load_4d(sb + kOffK + s * kTileBytes + kHalfBytes, km, bar(kBarKFull + s), 64, hk,
+                      kBN * t.j, b);
+          ++kiss;
+          if (!mbar_wait(bar(kBarVEmpty + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
+            raise_abort(abort_s, p.status);
+            break;
+          }
+          mbar_arrive_expect_tx(bar(kBarVFull + s), kTileBytes);
+          tma_load_4d(sb + kOffV + s * kTileBytes, &tm_v, bar(kBarVFull + s), 0, hk, kBN * t.j, b);
+          tma_load_4d(sb + kOffV + s * kTileBytes + kHalfBytes, &tm_v, bar(kBarVFull + s), 64,
+                      hk, kBN * t.j, b);
+          ++viss;
+          t.next();
+        }
+        // never leave with a copy in flight into this CTA's shared memory
+        for (int d = (kiss > kStages ? kiss - kStages : 0); d < kiss; ++d)
+          drain_wait(bar(kBarKFull + d % kStages), (d / kStages) & 1);
+        for (int d = (viss > kStages ? viss - kStages : 0); d < viss; ++d)
+          drain_wait(bar(kBarVFull + d % kStages), (d / kStages) & 1);
+      }
+      __syncwarp();
+    } else {
+      // ------------------------------------------------------- MMA issuer --
+      if (lane == 0) {
+        const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
+        const uint32_t idesc_pv = idesc_bf16_f32(kBM, kHD, 0, 1);
+        bool ok = mbar_wait(bar(kBarQFull), 0, abort_s, abort_g, kTimeoutNs);
+        tc_fence_after();
+        auto pv = [&](int tt) -> bool {
+          const int s = tt % kStages;
+          const uint32_t ph = (tt / kStages) & 1;
+          if (!mbar_wait(bar(kBarPFull), tt & 1, abort_s, abort_g, kTimeoutNs)) return false;
+          if (!mbar_wait(bar(kBarVFull + s), ph, abort_s, abort_g, kTimeoutNs)) return false;
+          tc_fence_after();
+          const uint32_t pa = sb + kOffP;
+          const uint32_t vb = sb + kOffV + s * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {  // 16 keys per step
+            const uint32_t a_off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+            const uint32_t b_off = kk * 2048;  // 16 key rows of 128 B
+            umma_bf16(tmem + kTmO, sdesc_sw128(pa + a_off, 16, 1024),
+                      sdesc_sw128(vb + b_off, kHalfBytes, 1024), idesc_pv,
+                      (tt > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(bar(kBarODone));
+          umma_commit(bar(kBarVEmpty + s));
+          return true;
+        };
+        PassIter t;
+        t.begin(qt, p.w);
+        int it = 0;
+        while (ok && !t.done()) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          const int sbuf = it & 1;
+          const uint32_t sph = (it >> 1) & 1;
+          if (!mbar_wait(bar(kBarKFull + s), ph, abort_s, abort_g, kTimeoutNs) ||
+              !mbar_wait(bar(kBarSFree + sbuf), sph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = sb + (t.kind() == kStd ? kOffQs : kOffQr);
+          const uint32_t b0 = sb + kOffK + s * kTileBytes;
+          const uint32_t d = tmem + (sbuf ? kTmS1 : kTmS0);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {  // 16 head dims per step
+            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+            umma_bf16(d, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(b0 + off, 16, 1024),
+                      idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar(kBarSFull + sbuf));
+          umma_commit(bar(kBarKEmpty + s));
+          if (it > 0 && !pv(it - 1)) {
+            ok = false;
+            break;
+          }
+          t.next();
+          ++it;
+        }
+        if (ok && it > 0) ok = pv(it - 1);
+        if (!ok) raise_abort(abort_s, p.status);
+        // every issued MMA retired before TMEM is released
+        umma_commit(bar(kBarDrain));
+        drain_wait(bar(kBarDrain), 0);
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [B, L, H, 128] bf16 -> 4-D map (dims innermost first: D, H, L, B), box of
+// 64 dims x 1 head x 128 rows, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap *m, const void *base, int B, int L, int H) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHD), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHD) * 2,
+                                 static_cast<cuuint64_t>(H) * kHD * 2,
+                                 static_cast<cuuint64_t>(L) * H * kHD * 2};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBN), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(bifocal_prefill_sm100_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  CUtensorMap mks, mkr, mv;
+  const void *krem = a.krem ? a.krem : a.kstd;
+  const void *kstd = a.kstd ? a.kstd : a.krem;
+  if (!make_map(&mks, kstd, a.B, a.L, a.Hkv) || !make_map(&mkr, krem, a.B, a.L, a.Hkv) ||
+      !make_map(&mv, a.v, a.B, a.L, a.Hkv))
+    return cudaErrorInvalidValue;
+  KParams p;
+  p.q = static_cast<const __nv_bfloat16 *>(a.q);
+  p.out = static_cast<__nv_bfloat16 *>(a.out);
+  p.lse = a.lse;
+  p.cs = a.table.cs;
+  p.status = a.status;
+  p.B = a.B;
+  p.L = a.L;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.G = a.G;
+  p.w = a.w_eff;
+  p.n_qtiles = (a.L + kBM - 1) / kBM;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * a.Hq;
+  bifocal_prefill_sm100_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(
+      mks, mkr, mv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace jl

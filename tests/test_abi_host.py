@@ -1,0 +1,130 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/jetlong.h declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "jetlong.h")
+
+FAKE = 0x10000  # an aligned non-null address; validation never dereferences it
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_attention_bifocal_b200 import build
+    build.build()
+    import long_context_attention_bifocal_b200 as jl
+    return jl.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(jl_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("jl_bifocal_prefill", "jl_bifocal_prefill_ex", "jl_bifocal_decode",
+              "jl_bifocal_decode_workspace_size", "jl_bifocal_prefill_workspace_size",
+              "jl_last_error", "jl_check_device_status", "jl_finalize", "jl_group_size"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in jetlong.h but not exported"
+
+
+def test_group_size_host(lib):
+    assert lib.jl_group_size(65536, 32768) == 2
+    assert lib.jl_group_size(131072, 32768) == 4
+    assert lib.jl_group_size(32768, 32768) == 1
+    assert lib.jl_group_size(98304, 32768) == 3
+    assert lib.jl_group_size(0, 5) == -1
+    assert lib.jl_group_size(5, 0) == -1
+
+
+def _prefill(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, B=1, L=256, Hq=4, Hkv=2, D=128,
+             w_local=64, w_pretrained=128, base=1e6, dtype=0, scale=0.0, flags=0,
+             ws=None, ws_bytes=0)
+    a.update(kw)
+    return lib.jl_bifocal_prefill_ex(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"],
+                                     a["L"], a["Hq"], a["Hkv"], a["D"], a["w_local"],
+                                     a["w_pretrained"], a["base"], a["dtype"], a["scale"],
+                                     a["flags"], a["ws"], a["ws_bytes"], None)
+
+
+INVALID, UNSUPPORTED = 1, 2
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=3, Hkv=2), INVALID),
+    (dict(B=0), INVALID),
+    (dict(L=0), INVALID),
+    (dict(D=7), INVALID),
+    (dict(D=64), UNSUPPORTED),            # bf16 path is head dim 128
+    (dict(D=256, dtype=1), UNSUPPORTED),  # fp32 path is 64 or 128
+    (dict(w_local=-1), INVALID),
+    (dict(w_pretrained=0), INVALID),
+    (dict(base=1.0), INVALID),
+    (dict(base=float("nan")), INVALID),
+    (dict(q=None), INVALID),
+    (dict(k=FAKE + 2), INVALID),          # misaligned
+    (dict(flags=1 << 7), INVALID),
+    (dict(dtype=5), INVALID),
+    (dict(ws=FAKE + 16, ws_bytes=1 << 30), INVALID),  # workspace not 256-aligned
+    (dict(ws=FAKE, ws_bytes=10), INVALID),            # workspace too small
+])
+def test_prefill_rejects(lib, kw, code):
+    assert _prefill(lib, **kw) == code
+    assert lib.jl_last_error()  # a message is left
+
+
+def _decode(lib, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, pos=100, cap=200, out=FAKE, lse=FAKE, ws=FAKE,
+             ws_bytes=1 << 30, B=1, Hq=8, Hkv=2, D=128, w_local=16, w_pretrained=64,
+             base=1e6, flags=0)
+    a.update(kw)
+    return lib.jl_bifocal_decode(a["q"], a["kc"], a["vc"], a["pos"], a["cap"], a["out"],
+                                 a["lse"], a["ws"], a["ws_bytes"], a["B"], a["Hq"],
+                                 a["Hkv"], a["D"], a["w_local"], a["w_pretrained"],
+                                 a["base"], a["flags"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(pos=200), INVALID),
+    (dict(pos=-1), INVALID),
+    (dict(Hq=6, Hkv=4), INVALID),
+    (dict(D=64), UNSUPPORTED),
+    (dict(ws=None), INVALID),
+    (dict(ws_bytes=8), INVALID),
+    (dict(kc=FAKE + 4), INVALID),
+    (dict(w_local=-3), INVALID),
+    (dict(flags=2), INVALID),
+])
+def test_decode_rejects(lib, kw, code):
+    assert _decode(lib, **kw) == code
+    assert lib.jl_last_error()
+
+
+def test_workspace_sizes(lib):
+    assert lib.jl_bifocal_prefill_workspace_size(1, 131072, 8, 128, 0) == 2 * 131072 * 8 * 128 * 2
+    assert lib.jl_bifocal_prefill_workspace_size(1, 100, 8, 64, 1) == 0
+    n = lib.jl_bifocal_decode_workspace_size(1, 32, 8, 128, 131071)
+    assert n > 0 and n % 4 == 0
+    assert lib.jl_bifocal_decode_workspace_size(1, 32, 8, 128, -1) == 0
+
+
+def test_product_path_has_no_oracle_or_fallback():
+    """The library package never imports the oracle and has no CPU path."""
+    pkg = os.path.join(ROOT, "long_context_attention_bifocal_b200")
+    for name in os.listdir(pkg):
+        if name.endswith(".py"):
+            src = open(os.path.join(pkg, name)).read()
+            assert "import oracle" not in src and "from oracle" not in src, name

@@ -1,0 +1,101 @@
+"""Bifocal decode on the GPU (through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import parity
+from long_context_attention_bifocal_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def run_decode(jl, q, kc, vc, pos, flags=0, **kw):
+    out, lse = jl.bifocal_decode(q.to(DEV), kc.to(DEV), vc.to(DEV), pos, flags=flags, **kw)
+    jl.check_device_status()
+    return out, lse
+
+
+def poison_tail(t, pos):
+    """NaN in every cache slot after pos: a kernel that reads them fails."""
+    t = t.clone()
+    t[:, pos + 1:] = float("nan")
+    return t
+
+
+@pytest.mark.parametrize("name", sorted(W.DECODE))
+def test_decode_full_size(jl, oracle_mod, name):
+    cfg = W.DECODE[name]
+    B, Hq, Hkv, D, n = cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["D"], cfg["n"]
+    pos = n - 1
+    cap = n + 64
+    q, kc, vc = W.decode_inputs(B, Hq, Hkv, D, cap, seed=cfg["seed"])
+    kc, vc = poison_tail(kc, pos), poison_tail(vc, pos)
+    kw = dict(w_local=cfg["w_local"], w_pretrained=cfg["w_pretrained"],
+              rope_base=cfg["rope_base"])
+    out, lse = run_decode(jl, q, kc, vc, pos, **kw)
+    ref_o, ref_l = oracle_mod.default().bifocal_decode(
+        W.to_oracle_array(q), W.to_oracle_array(kc[:, :pos + 1]),
+        W.to_oracle_array(vc[:, :pos + 1]), pos, **kw)
+    stats = parity.check(parity.to_np(out), parity.to_np(lse), ref_o, ref_l,
+                         max_abs=parity.BF16_MAX_ABS, mean_abs=parity.BF16_MEAN_ABS, what=name)
+    print(name, stats)
+    G = oracle_mod.default().group_size(n, cfg["w_pretrained"])
+    if G == 1:
+        out0, lse0 = run_decode(jl, q, kc, vc, pos, flags=jl.NO_BIFOCAL, **kw)
+        assert torch.equal(out, out0) and torch.equal(lse, lse0)
+
+
+EDGES = [
+    # (B, Hq, Hkv, pos, cap, w_local, w_pretrained)
+    (1, 8, 2, 0, 4, 16, 64),           # first token
+    (1, 8, 2, 1, 2, 16, 1),            # two tokens, G = 2
+    (1, 4, 4, 99, 128, 200, 30),       # every key local (pos < w_local), G = 4
+    (2, 8, 2, 5000, 6000, 0, 1000),    # every key remote, G = 6, B = 2
+    (1, 6, 3, 3001, 3100, 100, 1000),  # GQA 2, G = 4
+    (1, 3, 3, 4097, 5000, 64, 2048),   # GQA 1, G = 3
+    (3, 32, 8, 20000, 20001, 2048, 4096),  # B = 3, G = 5, full cache
+    (1, 16, 2, 777, 800, 5, 100),      # GQA 8 (two head groups per kv head)
+]
+
+
+@pytest.mark.parametrize("case", EDGES, ids=[f"B{c[0]}H{c[1]}x{c[2]}pos{c[3]}wl{c[5]}wp{c[6]}" for c in EDGES])
+def test_decode_edges(jl, oracle_mod, case):
+    B, Hq, Hkv, pos, cap, wl, wp = case
+    q, kc, vc = W.decode_inputs(B, Hq, Hkv, 128, cap, seed=pos + 3)
+    kc, vc = poison_tail(kc, pos), poison_tail(vc, pos)
+    kw = dict(w_local=wl, w_pretrained=wp, rope_base=1e6)
+    out, lse = run_decode(jl, q, kc, vc, pos, **kw)
+    ref_o, ref_l = oracle_mod.default().bifocal_decode(
+        W.to_oracle_array(q), W.to_oracle_array(kc[:, :pos + 1]),
+        W.to_oracle_array(vc[:, :pos + 1]), pos, **kw)
+    parity.check(parity.to_np(out), parity.to_np(lse), ref_o, ref_l,
+                 max_abs=parity.BF16_MAX_ABS, mean_abs=parity.BF16_MEAN_ABS, what=str(case))
+
+
+def test_decode_cache_is_not_written(jl):
+    q, kc, vc = W.decode_inputs(1, 8, 2, 128, 4000, seed=1)
+    kd, vd = kc.to(DEV), vc.to(DEV)
+    k0, v0 = kd.clone(), vd.clone()
+    jl.bifocal_decode(q.to(DEV), kd, vd, 3999, w_local=100, w_pretrained=1000, rope_base=1e6)
+    jl.check_device_status()
+    assert torch.equal(kd, k0) and torch.equal(vd, v0)
+
+
+def test_decode_matches_prefill_last_row(jl, oracle_mod):
+    """Decode at pos = L-1 over a cache of keys rotated at their original
+    positions equals the prefill row L-1 of the same sequence (same G)."""
+    L, Hq, Hkv = 3000, 8, 2
+    kw = dict(w_local=300, w_pretrained=1000, rope_base=1e6)
+    q, k, v = W.prefill_inputs(1, L, Hq, Hkv, 128, value_scale=1.0, seed=11)
+    out_p, lse_p = jl.bifocal_prefill(q.to(DEV), k.to(DEV), v.to(DEV), **kw)
+    orc = oracle_mod.default()
+    kf = k.float().numpy()
+    cache = np.stack([[orc.rope(kf[0, l, h].astype(np.float64), l, kw["rope_base"])
+                       for h in range(Hkv)] for l in range(L)])[None]
+    kc = torch.from_numpy(cache).to(torch.bfloat16)
+    out_d, lse_d = run_decode(jl, q[:, L - 1].contiguous(), kc, v, L - 1, **kw)
+    a, b = parity.to_np(out_d), parity.to_np(out_p[:, L - 1])
+    assert np.abs(a - b).max() <= parity.BF16_MAX_ABS
+    assert np.abs(parity.to_np(lse_d) - parity.to_np(lse_p[:, :, L - 1])).max() <= parity.LSE_ABS
