@@ -288,7 +288,7 @@ jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v, voi
   if (e != cudaSuccess) return cuda_fail(e, "key rotation launch");
   a.kstd = need_std ? kstd : nullptr;
   a.krem = need_rem ? krem : nullptr;
-  e = launch_prefill_sm100(a, s);
+  e = prefill_x2_supported(a) ? launch_prefill_sm100_x2(a, s) : launch_prefill_sm100(a, s);
   return e == cudaSuccess ? JL_OK : cuda_fail(e, "prefill launch");
 }
 

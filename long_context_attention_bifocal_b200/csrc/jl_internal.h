@@ -62,6 +62,9 @@ struct PrefillArgs {
 };
 
 cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s);
+// two query heads of one kv head per CTA; needs an even Hq / Hkv
+bool prefill_x2_supported(const PrefillArgs &a);
+cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_f32(const PrefillArgs &a, cudaStream_t s);
 
 struct DecodeArgs {

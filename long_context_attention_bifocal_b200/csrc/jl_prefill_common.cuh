@@ -1,0 +1,121 @@
+// jl_prefill_common.cuh -- pieces shared by the two tensor-core prefill
+// kernels: tile sizes, the pass schedule (the fused inclusion-exclusion merge
+// of Jet-Long, techwalker explainer §四 / bittide paper summary §3.2), the
+// 128-byte swizzle address, bounded waits and bf16 unpacking.
+#pragma once
+
+#include <climits>
+#include <cstdint>
+
+#include "jl_internal.h"
+#include "jl_sm100.cuh"
+
+namespace jl {
+namespace prefill {
+
+using namespace sm100;
+
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per tile
+constexpr int kHD = 128;  // head dim
+constexpr uint32_t kTileBytes = kBM * kHD * 2;  // one 128x128 bf16 tile
+constexpr uint32_t kHalfBytes = kTileBytes / 2;  // 64 columns (128 B rows)
+constexpr uint64_t kTimeoutNs = 1000000000ull;
+
+enum : int { kStd = 0, kRem = 1 };
+enum : int { kMaskNone = 0, kMaskFarOnly = 1, kMaskLocalOnly = 2 };
+
+// The pass schedule of query tile i.  Kv tile j <= i is at tile distance
+// d = i - j and spans pair distances [128d - 127, 128d + 127] (clipped at 0).
+// It holds a remote pair iff 128d + 127 >= w and a local pair iff
+// max(0, 128d - 127) < w.  The schedule runs two phases:
+//   remote phase: tiles 0..a (those holding a remote pair), K_rem and Q_rem,
+//                 masked to remote pairs where the tile also holds local ones;
+//   local phase:  tiles b..i (those holding a local pair), K_std and Q_std,
+//                 masked to local pairs where the tile also holds remote ones.
+// A tile straddling the window edge is visited once in each phase under
+// complementary masks; the diagonal tile also takes the causal mask.  The
+// online softmax does not depend on the order, and putting every remote pass
+// first lets a CTA keep one Q variant at a time.
+struct PassIter {
+  int i, w;      // query tile, local window (INT_MAX: every pair local)
+  int a, b;      // last tile with a remote pair (-1: none), first with a local pair
+  int phase;     // kRem, then kStd
+  int j;         // current kv tile
+
+  __device__ void begin(int qi, int wl) {
+    i = qi;
+    w = wl;
+    // smallest d with 128d + 127 >= w
+    const long long dmin = wl <= 127 ? 0 : (static_cast<long long>(wl) - 127 + kBN - 1) / kBN;
+    a = dmin > qi ? -1 : qi - static_cast<int>(dmin);
+    // largest d with 128d - 127 < w (none if w == 0)
+    if (wl <= 0) {
+      b = qi + 1;
+    } else {
+      const long long dmax = (static_cast<long long>(wl) + 126) / kBN;
+      b = dmax >= qi ? 0 : qi - static_cast<int>(dmax);
+    }
+    if (a >= 0) {
+      phase = kRem;
+      j = 0;
+    } else {
+      phase = kStd;
+      j = b;
+    }
+  }
+  __device__ bool done() const { return phase == kStd && j > i; }
+  __device__ int kind() const { return phase; }
+  __device__ int mask() const {
+    if (phase == kRem) return j >= b ? kMaskFarOnly : kMaskNone;
+    return j <= a ? kMaskLocalOnly : kMaskNone;
+  }
+  __device__ void next() {
+    ++j;
+    if (phase == kRem && j > a) {
+      phase = kStd;
+      j = b;
+    }
+  }
+};
+
+// byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled
+// [rows][128 B] tile (TMA SWIZZLE_128B and the UMMA descriptors agree on it)
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ void raise_abort(volatile int *abort_s, unsigned *status) {
+  *abort_s = 1;
+  atomicOr(status, kStatusTimeout);
+}
+
+// Wait used while draining: only the time limit ends it.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kTimeoutNs) break;
+  }
+}
+
+// mbar_wait for the softmax warps: the result is made uniform across the warp,
+// because the tcgen05.ld/st that follow a wait are warp-collective
+// (.sync.aligned) and must never run with part of the warp.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity,
+                                          const volatile int *abort_s,
+                                          const volatile unsigned *abort_g) {
+  const bool ok = mbar_wait(bar, parity, abort_s, abort_g, kTimeoutNs);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8]) {
+  const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    x[2 * j] = __uint_as_float(w4[j] << 16);
+    x[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
+  }
+}
+
+}  // namespace prefill
+}  // namespace jl

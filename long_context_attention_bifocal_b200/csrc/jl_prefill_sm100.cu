@@ -37,21 +37,17 @@
 #include <climits>
 #include <mutex>
 
-#include "jl_internal.h"
-#include "jl_sm100.cuh"
+#include "jl_prefill_common.cuh"
 
 namespace jl {
 namespace {
 
 using namespace sm100;
+using namespace prefill;
 
-constexpr int kBM = 128;  // query rows per tile
-constexpr int kBN = 128;  // keys per tile
-constexpr int kHD = 128;  // head dim
+// shared-memory layout (bytes from the 1 KiB-aligned base), barriers, TMEM
 constexpr int kStages = 2;
 constexpr int kThreads = 192;
-constexpr uint32_t kTileBytes = kBM * kHD * 2;  // one 128x128 bf16 tile
-constexpr uint32_t kHalfBytes = kTileBytes / 2;  // 64 columns (128 B rows)
 
 constexpr uint32_t kOffQs = 0;
 constexpr uint32_t kOffQr = kOffQs + kTileBytes;
@@ -83,53 +79,6 @@ static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmS0 = 0, kTmS1 = 128, kTmO = 256;
-constexpr uint64_t kTimeoutNs = 1000000000ull;
-
-enum : int { kStd = 0, kRem = 1 };
-enum : int { kMaskNone = 0, kMaskFarOnly = 1, kMaskLocalOnly = 2 };
-
-// The pass sequence of query tile i: for every kv tile j <= i, a remote pass
-// if the tile holds a remote pair, then a local pass if it holds a local pair.
-struct PassIter {
-  int i, w;        // query tile, local window (INT_MAX: every pair local)
-  int j, sub;      // current kv tile, 0/1 = first/second pass of the tile
-  bool two, far0;  // tile holds both classes; first pass is remote
-
-  __device__ bool has_far(int jj) const {
-    return static_cast<long long>(kBN) * (i - jj) + (kBN - 1) >= w;
-  }
-  __device__ bool has_local(int jj) const {
-    long long lo = static_cast<long long>(kBN) * (i - jj) - (kBM - 1);
-    if (lo < 0) lo = 0;
-    return lo < w;
-  }
-  __device__ void load() {
-    const bool f = has_far(j), l = has_local(j);
-    two = f && l;
-    far0 = f;
-  }
-  __device__ void begin(int qi, int wl) {
-    i = qi;
-    w = wl;
-    j = 0;
-    sub = 0;
-    load();
-  }
-  __device__ bool done() const { return j > i; }
-  __device__ int kind() const { return (sub == 0 && far0) ? kRem : kStd; }
-  __device__ int mask() const {
-    return two ? (sub == 0 ? kMaskFarOnly : kMaskLocalOnly) : kMaskNone;
-  }
-  __device__ void next() {
-    if (two && sub == 0) {
-      sub = 1;
-    } else {
-      ++j;
-      sub = 0;
-      if (j <= i) load();
-    }
-  }
-};
 
 struct KParams {
   const __nv_bfloat16 *q;
@@ -140,32 +89,6 @@ struct KParams {
   int B, L, Hq, Hkv, G, w, n_qtiles;
   float scale_log2;  // softmax scale * log2(e)
 };
-
-__device__ __forceinline__ uint32_t swz(int row, int chunk) {
-  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
-}
-
-__device__ __forceinline__ void raise_abort(volatile int *abort_s, unsigned *status) {
-  *abort_s = 1;
-  atomicOr(status, kStatusTimeout);
-}
-
-// Wait used while draining: only the time limit ends it.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kTimeoutNs) break;
-  }
-}
-
-__device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8]) {
-  const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    x[2 * j] = __uint_as_float(w4[j] << 16);
-    x[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
-  }
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
     bifocal_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_kstd,
@@ -275,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (!t.done()) {
         const int sbuf = it & 1;
         const uint32_t sph = (it >> 1) & 1;
-        if (!mbar_wait(bar(kBarSFull + sbuf), sph, abort_s, abort_g, kTimeoutNs)) {
+        if (!warp_wait(bar(kBarSFull + sbuf), sph, abort_s, abort_g)) {
           ok = false;
           break;
         }
@@ -331,12 +254,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (it > 0) {
           // PV of the previous pass done: P buffer free, O stable
-          if (!mbar_wait(bar(kBarODone), (it - 1) & 1, abort_s, abort_g, kTimeoutNs)) {
+          if (!warp_wait(bar(kBarODone), (it - 1) & 1, abort_s, abort_g)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if (resc && l > 0.f) {
+          // O rescale: the TMEM load/store is warp-collective, so the whole warp
+          // runs it when any row needs it (alpha is 1 for the other rows)
+          if (__any_sync(0xffffffffu, resc && l > 0.f)) {
+            if (!(resc && l > 0.f)) alpha = 1.f;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
               float o[32];
@@ -360,8 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         t.next();
         ++it;
       }
-      if (ok && !mbar_wait(bar(kBarODone), (it - 1) & 1, abort_s, abort_g, kTimeoutNs))
-        ok = false;
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok && !warp_wait(bar(kBarODone), (it - 1) & 1, abort_s, abort_g)) ok = false;
       if (!ok) {
         raise_abort(abort_s, p.status);
       } else {

@@ -1,0 +1,529 @@
+// jl_prefill_sm100_x2.cu -- bifocal prefill, two query heads per CTA.
+//
+// Same computation as jl_prefill_sm100.cu (Jet-Long, techwalker explainer
+// §二/§四, bittide paper summary §3.1-§3.2: local pairs at original positions,
+// remote pairs at f(x) = floor(x/G), merged by per-tile complementary-mask
+// passes inside one online softmax).  This kernel is the B200 throughput path
+// for grouped-query attention with an even group size: a CTA takes one
+// 128-row query tile of TWO query heads of the same kv head, so every K/V tile
+// it loads feeds two S = Q K^T and two O += P V products, and the tensor core
+// alternates between the two heads while each head's softmax runs.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax of head 0: thread r = query row r = TMEM lane r of S0/O0
+//   warps 4-7  softmax of head 1: the same on S1/O1
+//   warp 8     TMA producer: K tile (pre-rotated copy of the pass's class) and
+//              V tile into a 2-stage ring
+//   warp 9     TMEM allocation and every tcgen05.mma, from one thread
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.  After the
+// softmax has read S_t into registers it writes P_t (bf16, two per column) into
+// the first 64 columns of S_t, and O_t += P_t V takes P_t straight from TMEM;
+// the next S_t is issued only after that product has completed.
+//
+// Shared memory holds one Q variant per head: the remote passes of a query
+// tile all come before its local passes, so Q_rem is used first and is then
+// overwritten in place by Q_std (one switch per tile, signalled through the
+// q_ready barrier).  Q rotation runs in the softmax warps from the cos/sin
+// table; keys arrive already rotated.
+//
+// Exponentials: a fraction of each row's 2^x runs on the FMA pipe as
+// 2^floor(x) * p(x - floor(x)) with a cubic p fitted by least squares
+// (derive_exp2_poly.py, max relative error 1.1e-4), the rest on the MUFU unit,
+// so neither unit alone bounds the softmax.  Masked tiles use MUFU only.
+//
+// Every mbarrier wait is bounded; an abandoned wait raises the CTA abort flag
+// and the device status word, all roles drain their in-flight copies and MMAs,
+// TMEM is freed and the kernel returns.
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <mutex>
+
+#include "jl_prefill_common.cuh"
+
+namespace jl {
+namespace {
+
+using namespace sm100;
+using namespace prefill;
+
+constexpr int kStages = 2;
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+
+constexpr uint32_t kOffQ0 = 0;
+constexpr uint32_t kOffQ1 = kOffQ0 + kTileBytes;
+constexpr uint32_t kOffK = kOffQ1 + kTileBytes;
+constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+
+enum : int {
+  kBarQReady = 0,                  // [2] per head, 128 arrivals
+  kBarKFull = kBarQReady + 2,      // [kStages]
+  kBarKEmpty = kBarKFull + kStages,
+  kBarVFull = kBarKEmpty + kStages,
+  kBarVEmpty = kBarVFull + kStages,
+  kBarSFull = kBarVEmpty + kStages,  // [2] per head, tcgen05.commit
+  kBarPFull = kBarSFull + 2,         // [2] per head, 128 arrivals
+  kBarODone = kBarPFull + 2,         // [2] per head, tcgen05.commit
+  kBarDrain = kBarODone + 2,
+  kNumBars = kBarDrain + 1
+};
+
+constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
+constexpr uint32_t kOffSkip = kOffAbort + 4;
+constexpr uint32_t kSmemUsed = kOffSkip + 4;
+constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;
+static_assert(kSmemAlloc <= 232448, "shared memory budget");
+
+constexpr uint32_t kTmemCols = 512;
+__host__ __device__ constexpr uint32_t tm_s(int t) { return 128u * t; }
+__host__ __device__ constexpr uint32_t tm_o(int t) { return 256u + 128u * t; }
+
+// elements of each 32-column chunk whose 2^x runs on the FMA pipe
+constexpr int kPolyPer32 = 10;
+
+struct KParams {
+  const __nv_bfloat16 *q;
+  __nv_bfloat16 *out;
+  float *lse;
+  const float2 *cs;
+  unsigned *status;
+  int B, L, Hq, Hkv, G, w, n_qtiles;
+  float scale_log2;
+};
+
+// 2^x on the FMA pipe for x <= 8: 2^floor(x) times the cubic on the fraction.
+// Inputs below -127 are clamped (the result is then below 2^-126).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -127.f);
+  const float fl = floorf(x);
+  const float f = x - fl;
+  float p = fmaf(0.07816384732723236f, f, 0.22644174098968506f);
+  p = fmaf(p, f, 0.6953943967819214f);
+  p = fmaf(p, f, 1.0f);
+  const int e = static_cast<int>(fl);
+  return __int_as_float(__float_as_int(p) + static_cast<int>(static_cast<unsigned>(e) << 23));
+}
+
+// Rotates this thread's query row with the table at `pos` and writes it,
+// bf16 and swizzled, into the 128x128 tile at `dst`.
+__device__ __forceinline__ void rotate_q_row(uint8_t *dst, int r, const __nv_bfloat16 *qrow,
+                                             bool row_ok, const float2 *cs, int pos) {
+#pragma unroll 1
+  for (int c = 0; c < 8; ++c) {
+    float x1[8], x2[8];
+    if (row_ok) {
+      unpack8(*reinterpret_cast<const uint4 *>(qrow + 8 * c), x1);
+      unpack8(*reinterpret_cast<const uint4 *>(qrow + 64 + 8 * c), x2);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x1[e] = x2[e] = 0.f;
+    }
+    const float2 *t = cs + static_cast<int64_t>(pos) * 64 + 8 * c;
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 r0 = __ldg(t + 2 * e), r1 = __ldg(t + 2 * e + 1);
+      lo[e] = pack_bf16x2(x1[2 * e] * r0.x - x2[2 * e] * r0.y,
+                          x1[2 * e + 1] * r1.x - x2[2 * e + 1] * r1.y);
+      hi[e] = pack_bf16x2(x1[2 * e] * r0.y + x2[2 * e] * r0.x,
+                          x1[2 * e + 1] * r1.y + x2[2 * e + 1] * r1.x);
+    }
+    *reinterpret_cast<uint4 *>(dst + swz(r, c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *reinterpret_cast<uint4 *>(dst + kHalfBytes + swz(r, c)) =
+        make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bifocal_prefill_sm100_x2_kernel(const __grid_constant__ CUtensorMap tm_kstd,
+                                    const __grid_constant__ CUtensorMap tm_krem,
+                                    const __grid_constant__ CUtensorMap tm_v,
+                                    const KParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int pairs = p.Hq / 2;
+  const int bp = p.B * pairs;
+  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x / bp);
+  const int rem = static_cast<int>(blockIdx.x % bp);
+  const int hq0 = 2 * (rem % pairs);
+  const int b = rem / pairs;
+  const int hk = hq0 / (p.Hq / p.Hkv);
+
+  volatile int *abort_s = reinterpret_cast<volatile int *>(smem + kOffAbort);
+  volatile unsigned *abort_g = p.status;
+  auto bar = [&](int i) { return sb + kOffBar + 8u * static_cast<uint32_t>(i); };
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(kBarQReady + t), 128);
+      mbar_init(bar(kBarSFull + t), 1);
+      mbar_init(bar(kBarPFull + t), 128);
+      mbar_init(bar(kBarODone + t), 1);
+    }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
+    }
+    mbar_init(bar(kBarDrain), 1);
+    *abort_s = 0;
+    *reinterpret_cast<volatile int *>(smem + kOffSkip) = (*abort_g != 0u) ? 1 : 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(sb + kOffTmemSlot, kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + kOffTmemSlot);
+  const bool skip = *reinterpret_cast<volatile int *>(smem + kOffSkip) != 0;
+
+  if (!skip) {
+    if (warp < 8) {
+      // --------------------------------------------- softmax warpgroups --
+      const int t = warp >> 2;           // head of this warpgroup
+      const int r = threadIdx.x & 127;   // query row == TMEM lane
+      const int hq = hq0 + t;
+      const int qpos = kBM * qt + r;
+      const bool row_ok = qpos < p.L;
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+      const uint32_t s_col = lane_base + tm_s(t);
+      const uint32_t o_col = lane_base + tm_o(t);
+      uint8_t *qdst = smem + (t == 0 ? kOffQ0 : kOffQ1);
+      const __nv_bfloat16 *qrow =
+          p.q + ((static_cast<int64_t>(b) * p.L + (row_ok ? qpos : 0)) * p.Hq + hq) * kHD;
+      const int pos_std = row_ok ? qpos : 0;
+      const int pos_rem = row_ok ? qpos / p.G : 0;
+
+      PassIter it;
+      it.begin(qt, p.w);
+      // first Q variant = the class of the first pass
+      rotate_q_row(qdst, r, qrow, row_ok, p.cs, it.kind() == kRem ? pos_rem : pos_std);
+      fence_proxy_async_smem();
+      mbar_arrive(bar(kBarQReady + t));
+
+      float m = -INFINITY, l = 0.f;
+      int j = 0;
+      bool ok = true;
+      while (!it.done()) {
+        if (!warp_wait(bar(kBarSFull + t), j & 1, abort_s, abort_g)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(s_col + 32 * c, s + 32 * c);
+
+        const int kind = it.kind();
+        const int mk = it.mask();
+        const int kj = it.j;
+        it.next();
+        if (kind == kRem && !it.done() && it.kind() == kStd) {
+          // last remote pass of this tile: its S is complete, so Q may now be
+          // overwritten with the standard-position rotation
+          rotate_q_row(qdst, r, qrow, row_ok, p.cs, pos_std);
+          fence_proxy_async_smem();
+          mbar_arrive(bar(kBarQReady + t));
+        }
+
+        const bool causal = (kj == qt);
+        const bool plain = !causal && mk == kMaskNone;
+        float mt = -INFINITY;
+        if (plain) {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) {
+            s[e] *= p.scale_log2;
+            mt = fmaxf(mt, s[e]);
+          }
+        } else {
+          const int k0 = kBN * kj;
+#pragma unroll
+          for (int e = 0; e < 128; ++e) {
+            const int dd = qpos - (k0 + e);
+            bool valid = !causal || dd >= 0;
+            if (mk == kMaskFarOnly) valid = valid && dd >= p.w;
+            if (mk == kMaskLocalOnly) valid = valid && dd < p.w;
+            s[e] = valid ? s[e] * p.scale_log2 : -INFINITY;
+            mt = fmaxf(mt, s[e]);
+          }
+        }
+        const float m_new = fmaxf(m, mt);
+        float alpha = 1.f;
+        bool resc = false;
+        if (m_new > m + 8.f) {  // lazy rescale: only when the max grows by > 2^8
+          alpha = ex2_approx(m - m_new);
+          m = m_new;
+          resc = true;
+        }
+        // O_t is stable here: its last product was issued before this S and
+        // this S's completion covers it.  The TMEM access is warp-collective.
+        if (j > 0 && __any_sync(0xffffffffu, resc && l > 0.f)) {
+          const float a = (resc && l > 0.f) ? alpha : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(o_col + 32 * c, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= a;
+            tmem_st32(o_col + 32 * c, o);
+          }
+        }
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float x0 = s[32 * c + 2 * e] - mu;
+            const float x1 = s[32 * c + 2 * e + 1] - mu;
+            float p0, p1;
+            if (plain && 2 * e < kPolyPer32) {
+              p0 = exp2_poly(x0);
+              p1 = exp2_poly(x1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            rs += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(s_col + 16 * c, pk);
+        }
+        l = l * alpha + rs;
+        tc_fence_before();
+        mbar_arrive(bar(kBarPFull + t));
+        ++j;
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok && !warp_wait(bar(kBarODone + t), (j - 1) & 1, abort_s, abort_g)) ok = false;
+      if (!ok) {
+        raise_abort(abort_s, p.status);
+      } else {
+        tc_fence_after();
+        const float inv = 1.f / l;
+        __nv_bfloat16 *orow =
+            p.out + ((static_cast<int64_t>(b) * p.L + (row_ok ? qpos : 0)) * p.Hq + hq) * kHD;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32(o_col + 32 * c, o);
+          if (row_ok) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              uint4 w4;
+              w4.x = pack_bf16x2(o[8 * g + 0] * inv, o[8 * g + 1] * inv);
+              w4.y = pack_bf16x2(o[8 * g + 2] * inv, o[8 * g + 3] * inv);
+              w4.z = pack_bf16x2(o[8 * g + 4] * inv, o[8 * g + 5] * inv);
+              w4.w = pack_bf16x2(o[8 * g + 6] * inv, o[8 * g + 7] * inv);
+              *reinterpret_cast<uint4 *>(orow + 32 * c + 8 * g) = w4;
+            }
+          }
+        }
+        if (row_ok)
+          p.lse[(static_cast<int64_t>(b) * p.Hq + hq) * p.L + qpos] =
+              (m + __log2f(l)) * 0.69314718055994530942f;
+      }
+    } else if (warp == kProducerWarp) {
+      // ------------------------------------------------------ TMA producer --
+      if (lane == 0) {
+        prefetch_tmap(&tm_kstd);
+        prefetch_tmap(&tm_krem);
+        prefetch_tmap(&tm_v);
+        PassIter it;
+        it.begin(qt, p.w);
+        int kiss = 0, viss = 0;
+        while (!it.done()) {
+          const int s = kiss % kStages;
+          const uint32_t ph = (kiss / kStages) & 1;
+          if (!mbar_wait(bar(kBarKEmpty + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
+            raise_abort(abort_s, p.status);
+            break;
+          }
+          const CUtensorMap *km = it.kind() == kStd ? &tm_kstd : &tm_krem;
+          mbar_arrive_expect_tx(bar(kBarKFull + s), kTileBytes);
+          tma_load_4d(sb + kOffK + s * kTileBytes, km, bar(kBarKFull + s), 0, hk, kBN * it.j, b);
+          tma_load_4d(sb + kOffK + s * kTileBytes + kHalfBytes, km, bar(kBarKFull + s), 64, hk,
+                      kBN * it.j, b);
+          ++kiss;
+          if (!mbar_wait(bar(kBarVEmpty + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
+            raise_abort(abort_s, p.status);
+            break;
+          }
+          mbar_arrive_expect_tx(bar(kBarVFull + s), kTileBytes);
+          tma_load_4d(sb + kOffV + s * kTileBytes, &tm_v, bar(kBarVFull + s), 0, hk, kBN * it.j,
+                      b);
+          tma_load_4d(sb + kOffV + s * kTileBytes + kHalfBytes, &tm_v, bar(kBarVFull + s), 64,
+                      hk, kBN * it.j, b);
+          ++viss;
+          it.next();
+        }
+        for (int d = (kiss > kStages ? kiss - kStages : 0); d < kiss; ++d)
+          drain_wait(bar(kBarKFull + d % kStages), (d / kStages) & 1);
+        for (int d = (viss > kStages ? viss - kStages : 0); d < viss; ++d)
+          drain_wait(bar(kBarVFull + d % kStages), (d / kStages) & 1);
+      }
+      __syncwarp();
+    } else {
+      // ------------------------------------------------------- MMA issuer --
+      if (lane == 0) {
+        const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
+        const uint32_t idesc_pv = idesc_bf16_f32(kBM, kHD, 0, 1);
+        auto wait = [&](int i, uint32_t parity) {
+          return mbar_wait(bar(i), parity, abort_s, abort_g, kTimeoutNs);
+        };
+        PassIter it;
+        it.begin(qt, p.w);
+        bool ok = true;
+        int j = 0, qphase = 0;
+        int prev_kind = it.kind();
+        while (ok && !it.done()) {
+          const int kind = it.kind();
+          const int s = j % kStages;
+          const uint32_t ph = (j / kStages) & 1;
+          if (j == 0 || kind != prev_kind) {
+            // the Q variant this pass needs is in shared memory
+            ok = wait(kBarQReady + 0, qphase & 1) && wait(kBarQReady + 1, qphase & 1);
+            ++qphase;
+          }
+          ok = ok && wait(kBarKFull + s, ph);
+          if (!ok) break;
+          const uint32_t b0 = sb + kOffK + s * kTileBytes;
+          for (int t = 0; t < 2; ++t) {
+            // S_t holds P_t of the previous pass until that product completed
+            if (j > 0 && !wait(kBarODone + t, (j - 1) & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = sb + (t == 0 ? kOffQ0 : kOffQ1);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+              umma_bf16(tmem + tm_s(t), sdesc_sw128(a0 + off, 16, 1024),
+                        sdesc_sw128(b0 + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(bar(kBarSFull + t));
+          }
+          if (!ok) break;
+          umma_commit(bar(kBarKEmpty + s));
+          if (!wait(kBarVFull + s, ph)) {
+            ok = false;
+            break;
+          }
+          const uint32_t vb = sb + kOffV + s * kTileBytes;
+          for (int t = 0; t < 2; ++t) {
+            if (!wait(kBarPFull + t, j & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {  // 16 keys per step, P_t from TMEM
+              umma_bf16_ts(tmem + tm_o(t), tmem + tm_s(t) + 8 * kk,
+                           sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idesc_pv,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(bar(kBarODone + t));
+          }
+          if (!ok) break;
+          umma_commit(bar(kBarVEmpty + s));
+          prev_kind = kind;
+          it.next();
+          ++j;
+        }
+        if (!ok) raise_abort(abort_s, p.status);
+        umma_commit(bar(kBarDrain));
+        drain_wait(bar(kBarDrain), 0);
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap *m, const void *base, int B, int L, int H) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHD), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHD) * 2,
+                                 static_cast<cuuint64_t>(H) * kHD * 2,
+                                 static_cast<cuuint64_t>(L) * H * kHD * 2};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBN), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool prefill_x2_supported(const PrefillArgs &a) { return (a.Hq / a.Hkv) % 2 == 0; }
+
+cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(bifocal_prefill_sm100_x2_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  CUtensorMap mks, mkr, mv;
+  const void *krem = a.krem ? a.krem : a.kstd;
+  const void *kstd = a.kstd ? a.kstd : a.krem;
+  if (!make_map(&mks, kstd, a.B, a.L, a.Hkv) || !make_map(&mkr, krem, a.B, a.L, a.Hkv) ||
+      !make_map(&mv, a.v, a.B, a.L, a.Hkv))
+    return cudaErrorInvalidValue;
+  KParams p;
+  p.q = static_cast<const __nv_bfloat16 *>(a.q);
+  p.out = static_cast<__nv_bfloat16 *>(a.out);
+  p.lse = a.lse;
+  p.cs = a.table.cs;
+  p.status = a.status;
+  p.B = a.B;
+  p.L = a.L;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.G = a.G;
+  p.w = a.w_eff;
+  p.n_qtiles = (a.L + kBM - 1) / kBM;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * (a.Hq / 2);
+  bifocal_prefill_sm100_x2_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(
+      mks, mkr, mv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace jl
