@@ -135,6 +135,37 @@ jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped,
                             double rope_base, unsigned flags,
                             jl_stream_t stream);
 
+/*
+ * jl_bifocal_decode_noalloc -- the same single-token decode as
+ * jl_bifocal_decode, for callers that cannot allocate device memory: for
+ * example a host engine whose memory pool owns every device byte and forbids
+ * other allocations, or a latency-critical decode loop that cannot accept the
+ * implicit synchronisation an allocation brings.  This entry point has no
+ * counterpart in the paper; it is a packaging variant of the decode path.
+ *
+ *   Arguments, layouts and results are those of jl_bifocal_decode, without
+ *   the workspace.  It calls no cudaMalloc, cudaFree or other allocating
+ *   routine, and does not touch the library-owned angle table or status word:
+ *   the kernel evaluates its rotation angles itself (fp64 sincos rounded to
+ *   fp32, as the table holds them).
+ *   Split partials go to a fixed array compiled into the library:
+ *   1,048,576 floats (4 MiB), present on every GPU that loads the library until
+ *   the process exits.  Sizes are accepted while
+ *   B * Hq * n_splits * (D + 2) fits it (n_splits about 75 for B=1, Hq=32 at
+ *   pos = 131071); larger sizes return JL_ERR_UNSUPPORTED with a message.
+ *   The first call on each device looks up that array's device address (with
+ *   that device current) and caches it; make that first call before any stream
+ *   capture.  Every call shares the array and it keeps the last call's
+ *   partials; each call writes every entry it reads before reading it.  Calls
+ *   whose executions overlap on the GPU (other streams, other threads) race on
+ *   the array: serialise them.
+ */
+jl_status jl_bifocal_decode_noalloc(const void *q_new, const void *k_cache_roped,
+                                    const void *v_cache, int pos, int cache_capacity,
+                                    void *out, float *lse, int B, int Hq, int Hkv, int D,
+                                    int w_local, int w_pretrained, double rope_base,
+                                    unsigned flags, jl_stream_t stream);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 const char *jl_last_error(void);
 

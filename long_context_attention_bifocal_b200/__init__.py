@@ -16,6 +16,7 @@ import torch
 __all__ = [
     "NO_BIFOCAL", "JetLongError", "group_size", "bifocal_prefill",
     "prefill_workspace_size", "decode_workspace_size", "bifocal_decode",
+    "bifocal_decode_noalloc",
     "check_device_status", "finalize", "library_path", "load",
 ]
 
@@ -66,6 +67,8 @@ def load():
     L.jl_bifocal_decode.restype = i
     L.jl_bifocal_decode.argtypes = [p, p, p, i, i, p, p, p, sz, i, i, i, i, i, i, d,
                                     u, p]
+    L.jl_bifocal_decode_noalloc.restype = i
+    L.jl_bifocal_decode_noalloc.argtypes = [p, p, p, i, i, p, p, i, i, i, i, i, i, d, u, p]
     L.jl_last_error.restype = ctypes.c_char_p
     L.jl_last_error.argtypes = []
     L.jl_check_device_status.restype = i
@@ -176,6 +179,31 @@ def bifocal_decode(q_new, k_cache, v_cache, pos, *, w_local, w_pretrained, rope_
             _ptr(q_new), _ptr(k_cache), _ptr(v_cache), int(pos), cap, _ptr(out),
             _ptr(lse), _ptr(workspace), workspace.numel(), B, Hq, Hkv, D, int(w_local),
             int(w_pretrained), float(rope_base), int(flags), _stream(stream)))
+    return out, lse
+
+
+def bifocal_decode_noalloc(q_new, k_cache, v_cache, pos, *, w_local, w_pretrained,
+                           rope_base, out=None, lse=None, flags=0, stream=None):
+    """bifocal_decode without a workspace, for callers that cannot allocate
+    device memory: the library uses a fixed 4 MiB array of its own for the split
+    partials and allocates nothing (include/jetlong.h states the limits).  Passing
+    out/lse avoids the only allocations this wrapper would make."""
+    B, Hq, D = q_new.shape
+    cap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _need(q_new, "q_new", torch.bfloat16)
+    _need(k_cache, "k_cache", torch.bfloat16, (B, cap, Hkv, D))
+    _need(v_cache, "v_cache", torch.bfloat16, (B, cap, Hkv, D))
+    if out is None:
+        out = torch.empty_like(q_new)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q_new.device)
+    _need(out, "out", torch.bfloat16, (B, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq))
+    with torch.cuda.device(q_new.device):
+        _check(load().jl_bifocal_decode_noalloc(
+            _ptr(q_new), _ptr(k_cache), _ptr(v_cache), int(pos), cap, _ptr(out), _ptr(lse),
+            B, Hq, Hkv, D, int(w_local), int(w_pretrained), float(rope_base), int(flags),
+            _stream(stream)))
     return out, lse
 
 

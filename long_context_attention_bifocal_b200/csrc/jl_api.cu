@@ -366,6 +366,56 @@ jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped, const 
   return e == cudaSuccess ? JL_OK : cuda_fail(e, "decode launch");
 }
 
+jl_status jl_bifocal_decode_noalloc(const void *q_new, const void *k_cache_roped,
+                                    const void *v_cache, int pos, int cache_capacity,
+                                    void *out, float *lse, int B, int Hq, int Hkv, int D,
+                                    int w_local, int w_pretrained, double rope_base,
+                                    unsigned flags, jl_stream_t stream) {
+  g_last_error.clear();
+  jl_status st = check_common(B, 1, Hq, Hkv, D, w_local, w_pretrained, rope_base);
+  if (st != JL_OK) return st;
+  if (!q_new || !k_cache_roped || !v_cache || !out || !lse)
+    return fail(JL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q_new) || !aligned16(k_cache_roped) || !aligned16(v_cache) ||
+      !aligned16(out) || !aligned16(lse))
+    return fail(JL_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL)) != 0)
+    return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if (D != 128) return fail(JL_ERR_UNSUPPORTED, "decode supports head dim 128 (got %d)", D);
+  if (cache_capacity < 1 || pos < 0 || pos >= cache_capacity)
+    return fail(JL_ERR_INVALID_ARG, "need 0 <= pos (%d) < cache_capacity (%d)", pos,
+                cache_capacity);
+  const long long G = group_size_ll(static_cast<long long>(pos) + 1, w_pretrained);
+  const bool plain = (flags & JL_FLAG_NO_BIFOCAL) || G == 1;
+  DecodeArgs a;
+  a.q = static_cast<const __nv_bfloat16 *>(q_new);
+  a.kc = static_cast<const __nv_bfloat16 *>(k_cache_roped);
+  a.vc = static_cast<const __nv_bfloat16 *>(v_cache);
+  a.out = static_cast<__nv_bfloat16 *>(out);
+  a.lse = lse;
+  a.ws = nullptr;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.D = D;
+  a.pos = pos;
+  a.cap = cache_capacity;
+  a.G = static_cast<int>(G);
+  const long long fe = static_cast<long long>(pos) + 1 - w_local;
+  a.far_end = plain ? 0 : static_cast<int>(fe < 0 ? 0 : fe);
+  a.scale = static_cast<float>(1.0 / std::sqrt(D));
+  a.table = RopeTable{nullptr, 0, D / 2};
+  decode_plan(B, Hq, Hkv, pos, a.far_end, &a.chunk, &a.n_far_chunks, &a.n_chunks);
+  const size_t need = decode_ws_floats(B, Hq, D, a.n_chunks);
+  if (need > kDecodeNoAllocFloats)
+    return fail(JL_ERR_UNSUPPORTED,
+                "jl_bifocal_decode_noalloc: these sizes need %zu floats of scratch; its fixed "
+                "array holds %zu (use jl_bifocal_decode with a workspace)",
+                need, kDecodeNoAllocFloats);
+  cudaError_t e = launch_decode_noalloc(a, rope_base, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? JL_OK : cuda_fail(e, "no-alloc decode launch");
+}
+
 jl_status jl_check_device_status(jl_stream_t stream) {
   g_last_error.clear();
   DeviceState *d = nullptr;

@@ -23,6 +23,8 @@
 // Each CTA writes (o, m, l) for its chunk; a second kernel merges the chunks
 // with the same LogSumExp algebra the prefill uses and writes out and lse.
 #include <climits>
+#include <cmath>
+#include <mutex>
 
 #include "jl_internal.h"
 
@@ -58,9 +60,29 @@ struct SplitParams {
   float scale_log2;
 };
 
-template <int NH>
-__global__ void __launch_bounds__(kThreads)
-    bifocal_decode_split_kernel(const SplitParams p) {
+// theta_i = base^(-2i/D), computed on the host in fp64, for the variant that
+// evaluates its angles itself
+struct Thetas {
+  double t[kHalf];
+};
+
+// (cos, sin)(row * theta_pair) as fp32: read from the library's table, or, in
+// the table-free variant, evaluated here the same way the table was built
+// (fp64 sincos of the fp64 angle, rounded once).
+template <bool kSelfAngles>
+__device__ __forceinline__ float2 angle(const SplitParams &p, const double *theta, int64_t row,
+                                        int pair) {
+  if constexpr (kSelfAngles) {
+    double s, c;
+    sincos(static_cast<double>(row) * theta[pair], &s, &c);
+    return make_float2(static_cast<float>(c), static_cast<float>(s));
+  } else {
+    return p.cs[row * kHalf + pair];
+  }
+}
+
+template <int NH, bool kSelfAngles>
+__device__ __forceinline__ void decode_split_body(const SplitParams &p, const double *theta) {
   // cos/sin rows 0..63 as float4 [row][pair-pair e2][lane slot sl]:
   // (cos, sin) of pairs 8*sl + 2*e2 and 8*sl + 2*e2 + 1 -- 8 lanes of a key
   // read 128 contiguous bytes per load (32 KiB total)
@@ -89,8 +111,8 @@ __global__ void __launch_bounds__(kThreads)
   if (far) {
     for (int i = threadIdx.x; i < 64 * 4 * 8; i += kThreads) {
       const int row = i >> 5, e2 = (i >> 3) & 3, s8 = i & 7;
-      const float2 a = p.cs[row * kHalf + 8 * s8 + 2 * e2];
-      const float2 bq = p.cs[row * kHalf + 8 * s8 + 2 * e2 + 1];
+      const float2 a = angle<kSelfAngles>(p, theta, row, 8 * s8 + 2 * e2);
+      const float2 bq = angle<kSelfAngles>(p, theta, row, 8 * s8 + 2 * e2 + 1);
       tlo[i] = make_float4(a.x, a.y, bq.x, bq.y);
     }
   }
@@ -99,9 +121,7 @@ __global__ void __launch_bounds__(kThreads)
   // remote chunk) and pre-scaled by scale * log2(e).
   float q1[NH][8], q2[NH][8];
   {
-    const float2 *tp = p.cs + static_cast<int64_t>(p.pos) * kHalf + 8 * sl;
     const int udq = p.pos - p.pos / p.G;  // -dq >= 0
-    const float2 *tq = p.cs + static_cast<int64_t>(udq) * kHalf + 8 * sl;
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
       const __nv_bfloat16 *src = p.q + (static_cast<int64_t>(b) * p.Hq + h0 + h) * kD;
@@ -110,11 +130,11 @@ __global__ void __launch_bounds__(kThreads)
       unpack8(*reinterpret_cast<const uint4 *>(src + kHalf + 8 * sl), x2);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float2 a = tp[e];
+        const float2 a = angle<kSelfAngles>(p, theta, p.pos, 8 * sl + e);
         float y1 = x1[e] * a.x - x2[e] * a.y;
         float y2 = x1[e] * a.y + x2[e] * a.x;
         if (far) {  // rotate by dq = -udq: angle -udq*theta
-          const float2 r = tq[e];
+          const float2 r = angle<kSelfAngles>(p, theta, udq, 8 * sl + e);
           const float z1 = y1 * r.x + y2 * r.y;
           const float z2 = y2 * r.x - y1 * r.y;
           y1 = z1;
@@ -165,9 +185,9 @@ __global__ void __launch_bounds__(kThreads)
       const int u = kk - kk / p.G;
       const int hi = u >> 6, lo = u & 63;
       if (hi != hi_cached) {
-        const float2 *t = p.cs + static_cast<int64_t>(hi) * 64 * kHalf + 8 * sl;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) thi[e] = t[e];
+        for (int e = 0; e < 8; ++e)
+          thi[e] = angle<kSelfAngles>(p, theta, static_cast<int64_t>(hi) * 64, 8 * sl + e);
         hi_cached = hi;
       }
 #pragma unroll
@@ -283,6 +303,19 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+template <int NH>
+__global__ void __launch_bounds__(kThreads) bifocal_decode_split_kernel(const SplitParams p) {
+  decode_split_body<NH, false>(p, nullptr);
+}
+
+// The same split kernel with its angles evaluated in-kernel instead of read
+// from the library-owned table (used by the entry point that allocates nothing).
+template <int NH>
+__global__ void __launch_bounds__(kThreads)
+    bifocal_decode_split_selfangle_kernel(const SplitParams p, const Thetas th) {
+  decode_split_body<NH, true>(p, th.t);
+}
+
 // One CTA per (batch, query head): merges the chunk partials.
 __global__ void __launch_bounds__(kD)
     bifocal_decode_combine_kernel(const float *__restrict__ ws, __nv_bfloat16 *__restrict__ out,
@@ -313,7 +346,74 @@ cudaError_t launch_nh(const DecodeArgs &a, const SplitParams &sp, cudaStream_t s
   return cudaGetLastError();
 }
 
+template <int NH>
+cudaError_t launch_nh_selfangle(const DecodeArgs &a, const SplitParams &sp, const Thetas &th,
+                                cudaStream_t s) {
+  dim3 grid(a.n_chunks, a.Hkv * ((a.Hq / a.Hkv) / NH), a.B);
+  bifocal_decode_split_selfangle_kernel<NH><<<grid, kThreads, 0, s>>>(sp, th);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bifocal_decode_combine_kernel<<<a.B * a.Hq, kD, 0, s>>>(a.ws, a.out, a.lse, a.n_chunks);
+  return cudaGetLastError();
+}
+
+// Split partials of the entry point that allocates nothing: a fixed array in
+// the library's device image, present on every device that loads the library
+// until the process exits.  All such calls share it (the last call's partials
+// stay in it); every entry a call reads was written earlier by the same call.
+static __device__ __align__(256) float g_decode_noalloc_scratch[kDecodeNoAllocFloats];
+
+constexpr int kMaxScratchDevices = 64;
+
 }  // namespace
+
+// Device address of the fixed scratch array on the current device, resolved
+// once per device (with that device current) and cached.
+cudaError_t decode_noalloc_scratch(float **out) {
+  static std::mutex mu;
+  static float *addr[kMaxScratchDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_decode_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<float *>(ptr);
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_decode_noalloc(const DecodeArgs &a_in, double rope_base, cudaStream_t s) {
+  DecodeArgs a = a_in;
+  cudaError_t e = decode_noalloc_scratch(&a.ws);
+  if (e != cudaSuccess) return e;
+  Thetas th;
+  for (int i = 0; i < kHalf; ++i) th.t[i] = pow(rope_base, -2.0 * i / kD);
+  SplitParams sp;
+  sp.q = a.q;
+  sp.kc = a.kc;
+  sp.vc = a.vc;
+  sp.ws = a.ws;
+  sp.cs = nullptr;
+  sp.Hq = a.Hq;
+  sp.Hkv = a.Hkv;
+  sp.group = a.Hq / a.Hkv;
+  sp.pos = a.pos;
+  sp.cap = a.cap;
+  sp.G = a.G;
+  sp.far_end = a.far_end;
+  sp.chunk = a.chunk;
+  sp.n_far = a.n_far_chunks;
+  sp.n_chunks = a.n_chunks;
+  sp.scale_log2 = a.scale * 1.4426950408889634f;
+  if (sp.group % 4 == 0) return launch_nh_selfangle<4>(a, sp, th, s);
+  if (sp.group % 2 == 0) return launch_nh_selfangle<2>(a, sp, th, s);
+  return launch_nh_selfangle<1>(a, sp, th, s);
+}
 
 size_t decode_ws_floats(int B, int Hq, int D, int n_chunks) {
   return static_cast<size_t>(B) * Hq * n_chunks * (D + 2);

@@ -89,4 +89,10 @@ void decode_plan(int B, int Hq, int Hkv, int pos, int far_end, int *chunk,
                  int *n_far_chunks, int *n_chunks);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 
+// Fixed-size scratch of jl_bifocal_decode_noalloc, in floats (4 MiB).
+constexpr size_t kDecodeNoAllocFloats = static_cast<size_t>(1) << 20;
+// Same decode, split partials in the library's fixed scratch array and angles
+// evaluated in-kernel; a.ws is ignored.  Allocates nothing.
+cudaError_t launch_decode_noalloc(const DecodeArgs &a, double rope_base, cudaStream_t s);
+
 }  // namespace jl
