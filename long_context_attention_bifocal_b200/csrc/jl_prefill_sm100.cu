@@ -204,36 +204,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         float s[128];
-        {
-          const uint32_t col = lane_base + (sbuf ? kTmS1 : kTmS0);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(col + 32 * c, s + 32 * c);
-        }
+        tmem_ld128(lane_base + (sbuf ? kTmS1 : kTmS0), s);
         tc_fence_before();
         mbar_arrive(bar(kBarSFree + sbuf));
 
-        // scores in log2 units; masked entries -> -inf
+        // masked entries -> -inf; row max of the raw scores, 8 independent chains
         const int k0 = kBN * t.j;
         const int mk = t.mask();
         const bool causal = (t.j == qt);
-        float mt = -INFINITY;
-        if (!causal && mk == kMaskNone) {
-#pragma unroll
-          for (int e = 0; e < 128; ++e) {
-            s[e] *= p.scale_log2;
-            mt = fmaxf(mt, s[e]);
-          }
-        } else {
+        if (causal || mk != kMaskNone) {
 #pragma unroll
           for (int e = 0; e < 128; ++e) {
             const int dd = qpos - (k0 + e);
             bool valid = !causal || dd >= 0;
             if (mk == kMaskFarOnly) valid = valid && dd >= p.w;
             if (mk == kMaskLocalOnly) valid = valid && dd < p.w;
-            s[e] = valid ? s[e] * p.scale_log2 : -INFINITY;
-            mt = fmaxf(mt, s[e]);
+            s[e] = valid ? s[e] : -INFINITY;
           }
         }
+        float mx[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 128; ++e) mx[e & 7] = fmaxf(mx[e & 7], s[e]);
+        const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                         p.scale_log2;  // scale > 0 keeps the order
         const float m_new = fmaxf(m, mt);
         float alpha = 1.f;
         bool resc = false;
@@ -241,16 +237,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           alpha = ex2_approx(m - m_new);
           m = m_new;
           resc = true;
-        }
-        const float mu = (m == -INFINITY) ? 0.f : m;
-        float rs = 0.f;
-        uint32_t pk[64];
-#pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          const float p0 = ex2_approx(s[2 * e] - mu);
-          const float p1 = ex2_approx(s[2 * e + 1] - mu);
-          rs += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
         }
         if (it > 0) {
           // PV of the previous pass done: P buffer free, O stable
@@ -262,24 +248,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           // O rescale: the TMEM load/store is warp-collective, so the whole warp
           // runs it when any row needs it (alpha is 1 for the other rows)
           if (__any_sync(0xffffffffu, resc && l > 0.f)) {
-            if (!(resc && l > 0.f)) alpha = 1.f;
+            const float a = (resc && l > 0.f) ? alpha : 1.f;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
               float o[32];
               tmem_ld32(lane_base + kTmO + 32 * c, o);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] *= alpha;
+              for (int e = 0; e < 32; ++e) o[e] *= a;
               tmem_st32(lane_base + kTmO + 32 * c, o);
             }
           }
         }
-        l = l * alpha + rs;
+        // P = 2^(s * scale * log2(e) - m), one FFMA per element (-inf gives 0),
+        // stored as bf16 8 keys at a time into the swizzled P tile
+        const float neg_mu = (m == -INFINITY) ? 0.f : -m;
+        float rsum[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) rsum[a] = 0.f;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = ex2_approx(fmaf(s[8 * c + 2 * e], p.scale_log2, neg_mu));
+            const float p1 = ex2_approx(fmaf(s[8 * c + 2 * e + 1], p.scale_log2, neg_mu));
+            rsum[(2 * c + e) & 7] += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
           uint8_t *dst = smem + kOffP + (c >> 3) * kHalfBytes + swz(r, c & 7);
-          *reinterpret_cast<uint4 *>(dst) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
+        const float rs = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) +
+                         ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
+        l = l * alpha + rs;
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar(kBarPFull));

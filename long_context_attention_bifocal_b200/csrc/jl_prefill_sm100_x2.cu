@@ -222,10 +222,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        float s[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(s_col + 32 * c, s + 32 * c);
-
         const int kind = it.kind();
         const int mk = it.mask();
         const int kj = it.j;
@@ -240,24 +236,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         const bool causal = (kj == qt);
         const bool plain = !causal && mk == kMaskNone;
-        float mt = -INFINITY;
-        if (plain) {
+        const int k0 = kBN * kj;
+        // validity of column e for this row (only asked on masked tiles)
+        auto valid = [&](int e) {
+          const int dd = qpos - (k0 + e);
+          bool v = !causal || dd >= 0;
+          if (mk == kMaskFarOnly) v = v && dd >= p.w;
+          if (mk == kMaskLocalOnly) v = v && dd < p.w;
+          return v;
+        };
+        // pass 1 over S: row max of the raw scores, 8 independent chains
+        float mt;
+        {
+          float sv[128];
+          tmem_ld128(s_col, sv);
+          float mx[8];
 #pragma unroll
-          for (int e = 0; e < 128; ++e) {
-            s[e] *= p.scale_log2;
-            mt = fmaxf(mt, s[e]);
-          }
-        } else {
-          const int k0 = kBN * kj;
+          for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
+          if (plain) {
 #pragma unroll
-          for (int e = 0; e < 128; ++e) {
-            const int dd = qpos - (k0 + e);
-            bool valid = !causal || dd >= 0;
-            if (mk == kMaskFarOnly) valid = valid && dd >= p.w;
-            if (mk == kMaskLocalOnly) valid = valid && dd < p.w;
-            s[e] = valid ? s[e] * p.scale_log2 : -INFINITY;
-            mt = fmaxf(mt, s[e]);
+            for (int e = 0; e < 128; ++e) mx[e & 7] = fmaxf(mx[e & 7], sv[e]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 128; ++e)
+              mx[e & 7] = fmaxf(mx[e & 7], valid(e) ? sv[e] : -INFINITY);
           }
+          mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+               p.scale_log2;  // scale > 0 keeps the order
         }
         const float m_new = fmaxf(m, mt);
         float alpha = 1.f;
@@ -280,15 +286,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(o_col + 32 * c, o);
           }
         }
-        const float mu = (m == -INFINITY) ? 0.f : m;
-        float rs = 0.f;
+        // pass 2 over S, 32 columns at a time: P = 2^(s * scale * log2(e) - m),
+        // written as bf16 into columns of S that are already consumed
+        const float neg_mu = (m == -INFINITY) ? 0.f : -m;
+        float rsum[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) rsum[a] = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
+          float sv[32];
+          tmem_ld32(s_col + 32 * c, sv);
+          if (!plain) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sv[e] = valid(32 * c + e) ? sv[e] : -INFINITY;
+          }
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float x0 = s[32 * c + 2 * e] - mu;
-            const float x1 = s[32 * c + 2 * e + 1] - mu;
+            const float x0 = fmaf(sv[2 * e], p.scale_log2, neg_mu);
+            const float x1 = fmaf(sv[2 * e + 1], p.scale_log2, neg_mu);
             float p0, p1;
             if (plain && 2 * e < kPolyPer32) {
               p0 = exp2_poly(x0);
@@ -297,11 +313,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               p0 = ex2_approx(x0);
               p1 = ex2_approx(x1);
             }
-            rs += p0 + p1;
+            rsum[e & 7] += p0 + p1;
             pk[e] = pack_bf16x2(p0, p1);
           }
           tmem_st16(s_col + 16 * c, pk);
         }
+        const float rs = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) +
+                         ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
         l = l * alpha + rs;
         tc_fence_before();
         mbar_arrive(bar(kBarPFull + t));
