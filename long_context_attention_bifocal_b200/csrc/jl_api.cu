@@ -308,10 +308,13 @@ jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v, void *
 
 size_t jl_bifocal_decode_workspace_size(int B, int Hq, int Hkv, int D, int pos) {
   if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || pos < 0 || Hq % Hkv != 0) return 0;
-  // the remote/local split adds at most one chunk
+  // the remote/local split adds at most one chunk to either plan
   int chunk = 0, n_far = 0, n_chunks = 0;
   decode_plan(B, Hq, Hkv, pos, 0, &chunk, &n_far, &n_chunks);
-  return decode_ws_floats(B, Hq, D, n_chunks + 1) * sizeof(float);
+  int chunk2 = 0, n_far2 = 0, n_chunks2 = 0;
+  decode_mma_plan(B, pos, 0, &chunk2, &n_far2, &n_chunks2);
+  const int most = n_chunks > n_chunks2 ? n_chunks : n_chunks2;
+  return decode_ws_floats(B, Hq, D, most + 1) * sizeof(float);
 }
 
 jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped, const void *v_cache,
@@ -359,10 +362,19 @@ jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped, const 
   const long long fe = static_cast<long long>(pos) + 1 - w_local;
   a.far_end = plain ? 0 : static_cast<int>(fe < 0 ? 0 : fe);
   a.scale = static_cast<float>(1.0 / std::sqrt(D));
-  decode_plan(B, Hq, Hkv, pos, a.far_end, &a.chunk, &a.n_far_chunks, &a.n_chunks);
   st = rope_table(D, rope_base, pos + 1 < 64 ? 64 : pos + 1, s, &a.table);
   if (st != JL_OK) return st;
-  cudaError_t e = launch_decode(a, s);
+  cudaError_t e;
+  if (decode_mma_supported(Hq, Hkv, D)) {
+    unsigned *status = nullptr;
+    st = status_word(&status);
+    if (st != JL_OK) return st;
+    decode_mma_plan(B, pos, a.far_end, &a.chunk, &a.n_far_chunks, &a.n_chunks);
+    e = launch_decode_mma(a, status, s);
+  } else {
+    decode_plan(B, Hq, Hkv, pos, a.far_end, &a.chunk, &a.n_far_chunks, &a.n_chunks);
+    e = launch_decode(a, s);
+  }
   return e == cudaSuccess ? JL_OK : cuda_fail(e, "decode launch");
 }
 

@@ -415,6 +415,11 @@ cudaError_t launch_decode_noalloc(const DecodeArgs &a_in, double rope_base, cuda
   return launch_nh_selfangle<1>(a, sp, th, s);
 }
 
+cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t s) {
+  bifocal_decode_combine_kernel<<<a.B * a.Hq, kD, 0, s>>>(a.ws, a.out, a.lse, a.n_chunks);
+  return cudaGetLastError();
+}
+
 size_t decode_ws_floats(int B, int Hq, int D, int n_chunks) {
   return static_cast<size_t>(B) * Hq * n_chunks * (D + 2);
 }

@@ -88,6 +88,14 @@ size_t decode_ws_floats(int B, int Hq, int D, int n_chunks);
 void decode_plan(int B, int Hq, int Hkv, int pos, int far_end, int *chunk,
                  int *n_far_chunks, int *n_chunks);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+// merges a.n_chunks split partials of a.ws into a.out and a.lse
+cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t s);
+
+// TMA-staged tensor-core decode (all kv heads of a key chunk per CTA):
+// needs D == 128, Hkv <= 8 and Hq / Hkv <= 16.
+bool decode_mma_supported(int Hq, int Hkv, int D);
+void decode_mma_plan(int B, int pos, int far_end, int *chunk, int *n_far, int *n_chunks);
+cudaError_t launch_decode_mma(const DecodeArgs &a, unsigned *status, cudaStream_t s);
 
 // Fixed-size scratch of jl_bifocal_decode_noalloc, in floats (4 MiB).
 constexpr size_t kDecodeNoAllocFloats = static_cast<size_t>(1) << 20;

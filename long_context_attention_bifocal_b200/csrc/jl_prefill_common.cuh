@@ -117,5 +117,24 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8]) {
   }
 }
 
+// 2^x on the FMA/ALU pipes instead of the MUFU unit, for x <= 8:
+// 2^floor(x) * p(x - floor(x)) with a cubic p fitted by weighted least squares
+// on Chebyshev nodes with p(0) = 1 and p(1) = 2 (derive_exp2_poly.py; maximum
+// relative error 1.1e-4, below the bf16 rounding of P that follows).
+// floor(x) comes from one round-down add of 1.5 * 2^23, after which the low
+// mantissa bits hold floor(x) as an integer -- no float-to-int conversion.
+// Inputs below -127 are clamped (the result is then below 2^-126).
+__device__ __forceinline__ float exp2_poly(float x) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  x = fmaxf(x, -127.f);
+  const float t = __fadd_rd(x, kMagic);  // kMagic + floor(x), exact
+  const float f = x - (t - kMagic);      // fraction in [0, 1)
+  const int e = __float_as_int(t) - __float_as_int(kMagic);  // floor(x)
+  float p = fmaf(0.07816384732723236f, f, 0.22644174098968506f);
+  p = fmaf(p, f, 0.6953943967819214f);
+  p = fmaf(p, f, 1.0f);
+  return __int_as_float(__float_as_int(p) + static_cast<int>(static_cast<unsigned>(e) << 23));
+}
+
 }  // namespace prefill
 }  // namespace jl

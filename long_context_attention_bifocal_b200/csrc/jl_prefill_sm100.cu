@@ -19,11 +19,16 @@
 //
 // B200 design: one CTA per (batch, query head, 128-row query tile), heaviest
 // tiles first.  Warp roles:
-//   warps 0-3  rotate the Q tile twice (standard and remapped) into swizzled
-//              shared memory, then run the online softmax: thread r owns query
-//              row r = TMEM lane r, reads S from TMEM, writes P (bf16) to shared
-//              memory, rescales O in TMEM when the running max grows by more
-//              than 2^8 (lazy rescale), and finally normalises O and stores it.
+//   warps 0-3  rotate the Q tile into swizzled shared memory (remapped
+//              positions for the remote passes, then, once they are done,
+//              standard positions for the local passes), and run the online
+//              softmax: thread r owns query row r = TMEM lane r, reads S from
+//              TMEM, writes P (bf16) into one of two shared-memory buffers,
+//              rescales O in TMEM when the running max grows by more than 2^8
+//              (lazy rescale), and finally normalises O and stores it.  Part of
+//              each row's exponentials run on the FMA pipe (exp2_poly).
+//              With P double-buffered the softmax of pass j+1 overlaps the
+//              product O += P V of pass j.
 //   warp 4     TMA producer: K tile (pre-rotated copy of the needed class) and
 //              V tile per pass into a 2-stage ring.
 //   warp 5     allocates TMEM and issues every tcgen05.mma from one thread:
@@ -49,24 +54,23 @@ using namespace prefill;
 constexpr int kStages = 2;
 constexpr int kThreads = 192;
 
-constexpr uint32_t kOffQs = 0;
-constexpr uint32_t kOffQr = kOffQs + kTileBytes;
-constexpr uint32_t kOffK = kOffQr + kTileBytes;
+constexpr uint32_t kOffQ = 0;  // the Q variant of the current phase
+constexpr uint32_t kOffK = kOffQ + kTileBytes;
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
-constexpr uint32_t kOffP = kOffV + kStages * kTileBytes;
-constexpr uint32_t kOffBar = kOffP + kTileBytes;
+constexpr uint32_t kOffP = kOffV + kStages * kTileBytes;  // [2] P buffers
+constexpr uint32_t kOffBar = kOffP + 2 * kTileBytes;
 
 enum : int {
-  kBarQFull = 0,
+  kBarQFull = 0,  // phase 0: first Q variant; phase 1: Q_std after the remote passes
   kBarKFull = 1,
   kBarKEmpty = kBarKFull + kStages,
   kBarVFull = kBarKEmpty + kStages,
   kBarVEmpty = kBarVFull + kStages,
   kBarSFull = kBarVEmpty + kStages,
   kBarSFree = kBarSFull + 2,
-  kBarPFull = kBarSFree + 2,
-  kBarODone = kBarPFull + 1,
-  kBarDrain = kBarODone + 1,
+  kBarPFull = kBarSFree + 2,  // [2] per P buffer
+  kBarODone = kBarPFull + 2,  // [2] per P buffer: O += P V of that buffer done
+  kBarDrain = kBarODone + 2,
   kNumBars = kBarDrain + 1
 };
 
@@ -79,6 +83,12 @@ static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmS0 = 0, kTmS1 = 128, kTmO = 256;
+
+// pairs (of each 4 in an 8-key chunk) whose 2^x runs on the FMA pipe
+#ifndef JL_POLY_PAIRS
+#define JL_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = JL_POLY_PAIRS;
 
 struct KParams {
   const __nv_bfloat16 *q;
@@ -124,9 +134,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarSFull + s), 1);
       mbar_init(bar(kBarSFree + s), 128);
+      mbar_init(bar(kBarPFull + s), 128);
+      mbar_init(bar(kBarODone + s), 1);
     }
-    mbar_init(bar(kBarPFull), 128);
-    mbar_init(bar(kBarODone), 1);
     mbar_init(bar(kBarDrain), 1);
     *abort_s = 0;
     *reinterpret_cast<volatile int *>(smem + kOffSkip) = (*abort_g != 0u) ? 1 : 0;
@@ -148,14 +158,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qpos = kBM * qt + r;
       const bool row_ok = qpos < p.L;
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
-      const bool need_rem = p.w != INT_MAX;
-
-      // Q_std = R(q) Q and Q_rem = R(f(q)) Q, bf16, in the swizzled K-major
-      // layout the UMMA descriptors expect (two 64-column halves).
-      {
-        const int pr = qpos / p.G;
-        const __nv_bfloat16 *qrow =
-            p.q + ((static_cast<int64_t>(b) * p.L + (row_ok ? qpos : 0)) * p.Hq + hq) * kHD;
+      const __nv_bfloat16 *qrow =
+          p.q + ((static_cast<int64_t>(b) * p.L + (row_ok ? qpos : 0)) * p.Hq + hq) * kHD;
+      const int pos_std = row_ok ? qpos : 0;
+      const int pos_rem = row_ok ? qpos / p.G : 0;
+      // Q rotated at `pos`, bf16, in the swizzled K-major layout the UMMA
+      // descriptors expect (two 64-column halves)
+      auto rotate_q = [&](int pos) {
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           float x1[8], x2[8];
@@ -166,29 +175,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) x1[e] = x2[e] = 0.f;
           }
+          const float2 *tb = p.cs + static_cast<int64_t>(pos) * 64 + 8 * c;
+          uint32_t lo[4], hi[4];
 #pragma unroll
-          for (int pass = 0; pass < 2; ++pass) {
-            if (pass == 1 && !need_rem) break;
-            const int pos = row_ok ? (pass == 0 ? qpos : pr) : 0;
-            const float2 *t = p.cs + static_cast<int64_t>(pos) * 64 + 8 * c;
-            uint32_t lo[4], hi[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 r0 = __ldg(t + 2 * e), r1 = __ldg(t + 2 * e + 1);
-              lo[e] = pack_bf16x2(x1[2 * e] * r0.x - x2[2 * e] * r0.y,
-                                  x1[2 * e + 1] * r1.x - x2[2 * e + 1] * r1.y);
-              hi[e] = pack_bf16x2(x1[2 * e] * r0.y + x2[2 * e] * r0.x,
-                                  x1[2 * e + 1] * r1.y + x2[2 * e + 1] * r1.x);
-            }
-            uint8_t *dst = smem + (pass == 0 ? kOffQs : kOffQr);
-            *reinterpret_cast<uint4 *>(dst + swz(r, c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            *reinterpret_cast<uint4 *>(dst + kHalfBytes + swz(r, c)) =
-                make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          for (int e = 0; e < 4; ++e) {
+            const float2 r0 = __ldg(tb + 2 * e), r1 = __ldg(tb + 2 * e + 1);
+            lo[e] = pack_bf16x2(x1[2 * e] * r0.x - x2[2 * e] * r0.y,
+                                x1[2 * e + 1] * r1.x - x2[2 * e + 1] * r1.y);
+            hi[e] = pack_bf16x2(x1[2 * e] * r0.y + x2[2 * e] * r0.x,
+                                x1[2 * e + 1] * r1.y + x2[2 * e + 1] * r1.x);
           }
+          uint8_t *dst = smem + kOffQ;
+          *reinterpret_cast<uint4 *>(dst + swz(r, c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint4 *>(dst + kHalfBytes + swz(r, c)) =
+              make_uint4(hi[0], hi[1], hi[2], hi[3]);
         }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(kBarQFull));
+      };
+      {
+        PassIter t0;
+        t0.begin(qt, p.w);
+        rotate_q(t0.kind() == kRem ? pos_rem : pos_std);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(bar(kBarQFull));
 
       float m = -INFINITY, l = 0.f;
       PassIter t;
@@ -208,10 +217,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(kBarSFree + sbuf));
 
-        // masked entries -> -inf; row max of the raw scores, 8 independent chains
         const int k0 = kBN * t.j;
         const int mk = t.mask();
         const bool causal = (t.j == qt);
+        const int kind = t.kind();
+        t.next();
+        if (kind == kRem && !t.done() && t.kind() == kStd)
+          rotate_q(pos_std);  // last remote pass: its S is complete, Q may change
+        // masked entries -> -inf; row max of the raw scores, 8 independent chains
         if (causal || mk != kMaskNone) {
 #pragma unroll
           for (int e = 0; e < 128; ++e) {
@@ -238,57 +251,71 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_new;
           resc = true;
         }
-        if (it > 0) {
-          // PV of the previous pass done: P buffer free, O stable
-          if (!warp_wait(bar(kBarODone), (it - 1) & 1, abort_s, abort_g)) {
+        const int pbuf = it & 1;
+        // O rescale (rare) needs the product of pass it-1 complete.  Waits on a
+        // per-buffer barrier are unambiguous: the product of pass it-3 is done
+        // (this pass's S completed after it) and pass it+1's cannot start.
+        // The TMEM access is warp-collective.
+        if (it > 0 && __any_sync(0xffffffffu, resc && l > 0.f)) {
+          if (!warp_wait(bar(kBarODone + ((it - 1) & 1)), ((it - 1) >> 1) & 1, abort_s,
+                         abort_g)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          // O rescale: the TMEM load/store is warp-collective, so the whole warp
-          // runs it when any row needs it (alpha is 1 for the other rows)
-          if (__any_sync(0xffffffffu, resc && l > 0.f)) {
-            const float a = (resc && l > 0.f) ? alpha : 1.f;
+          const float a = (resc && l > 0.f) ? alpha : 1.f;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              float o[32];
-              tmem_ld32(lane_base + kTmO + 32 * c, o);
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(lane_base + kTmO + 32 * c, o);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] *= a;
-              tmem_st32(lane_base + kTmO + 32 * c, o);
-            }
+            for (int e = 0; e < 32; ++e) o[e] *= a;
+            tmem_st32(lane_base + kTmO + 32 * c, o);
           }
         }
         // P = 2^(s * scale * log2(e) - m), one FFMA per element (-inf gives 0),
-        // stored as bf16 8 keys at a time into the swizzled P tile
+        // stored as bf16 8 keys at a time into P buffer it & 1; that buffer was
+        // last read by the product of pass it-2, complete before this S.
+        const bool plain = !causal && mk == kMaskNone;
         const float neg_mu = (m == -INFINITY) ? 0.f : -m;
         float rsum[8];
 #pragma unroll
         for (int a = 0; a < 8; ++a) rsum[a] = 0.f;
+        uint8_t *pdst = smem + kOffP + pbuf * kTileBytes;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           uint32_t pk[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p0 = ex2_approx(fmaf(s[8 * c + 2 * e], p.scale_log2, neg_mu));
-            const float p1 = ex2_approx(fmaf(s[8 * c + 2 * e + 1], p.scale_log2, neg_mu));
+            const float x0 = fmaf(s[8 * c + 2 * e], p.scale_log2, neg_mu);
+            const float x1 = fmaf(s[8 * c + 2 * e + 1], p.scale_log2, neg_mu);
+            float p0, p1;
+            if (plain && e < kPolyPairs) {
+              p0 = exp2_poly(x0);
+              p1 = exp2_poly(x1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
             rsum[(2 * c + e) & 7] += p0 + p1;
             pk[e] = pack_bf16x2(p0, p1);
           }
-          uint8_t *dst = smem + kOffP + (c >> 3) * kHalfBytes + swz(r, c & 7);
-          *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4 *>(pdst + (c >> 3) * kHalfBytes + swz(r, c & 7)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
         const float rs = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) +
                          ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
         l = l * alpha + rs;
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(bar(kBarPFull));
-        t.next();
+        mbar_arrive(bar(kBarPFull + pbuf));
         ++it;
       }
       ok = __all_sync(0xffffffffu, ok);
-      if (ok && !warp_wait(bar(kBarODone), (it - 1) & 1, abort_s, abort_g)) ok = false;
+      // the last product (in-order completion: every earlier one is done too)
+      if (ok && !warp_wait(bar(kBarODone + ((it - 1) & 1)), ((it - 1) >> 1) & 1, abort_s,
+                           abort_g))
+        ok = false;
       if (!ok) {
         raise_abort(abort_s, p.status);
       } else {
@@ -361,15 +388,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
         const uint32_t idesc_pv = idesc_bf16_f32(kBM, kHD, 0, 1);
-        bool ok = mbar_wait(bar(kBarQFull), 0, abort_s, abort_g, kTimeoutNs);
-        tc_fence_after();
+        bool ok = true;
         auto pv = [&](int tt) -> bool {
           const int s = tt % kStages;
           const uint32_t ph = (tt / kStages) & 1;
-          if (!mbar_wait(bar(kBarPFull), tt & 1, abort_s, abort_g, kTimeoutNs)) return false;
+          const int pbuf = tt & 1;
+          if (!mbar_wait(bar(kBarPFull + pbuf), (tt >> 1) & 1, abort_s, abort_g, kTimeoutNs))
+            return false;
           if (!mbar_wait(bar(kBarVFull + s), ph, abort_s, abort_g, kTimeoutNs)) return false;
           tc_fence_after();
-          const uint32_t pa = sb + kOffP;
+          const uint32_t pa = sb + kOffP + pbuf * kTileBytes;
           const uint32_t vb = sb + kOffV + s * kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {  // 16 keys per step
@@ -379,14 +407,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                       sdesc_sw128(vb + b_off, kHalfBytes, 1024), idesc_pv,
                       (tt > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(bar(kBarODone));
+          umma_commit(bar(kBarODone + pbuf));
           umma_commit(bar(kBarVEmpty + s));
           return true;
         };
         PassIter t;
         t.begin(qt, p.w);
-        int it = 0;
+        int it = 0, qphase = 0, prev_kind = t.kind();
         while (ok && !t.done()) {
+          const int kind = t.kind();
+          if (it == 0 || kind != prev_kind) {
+            // the Q variant this pass needs is in shared memory
+            ok = mbar_wait(bar(kBarQFull), qphase & 1, abort_s, abort_g, kTimeoutNs);
+            ++qphase;
+            if (!ok) break;
+          }
+          prev_kind = kind;
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
           const int sbuf = it & 1;
@@ -397,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = sb + (t.kind() == kStd ? kOffQs : kOffQr);
+          const uint32_t a0 = sb + kOffQ;
           const uint32_t b0 = sb + kOffK + s * kTileBytes;
           const uint32_t d = tmem + (sbuf ? kTmS1 : kTmS0);
 #pragma unroll

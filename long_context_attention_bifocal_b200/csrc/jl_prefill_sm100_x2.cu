@@ -95,19 +95,6 @@ struct KParams {
   float scale_log2;
 };
 
-// 2^x on the FMA pipe for x <= 8: 2^floor(x) times the cubic on the fraction.
-// Inputs below -127 are clamped (the result is then below 2^-126).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -127.f);
-  const float fl = floorf(x);
-  const float f = x - fl;
-  float p = fmaf(0.07816384732723236f, f, 0.22644174098968506f);
-  p = fmaf(p, f, 0.6953943967819214f);
-  p = fmaf(p, f, 1.0f);
-  const int e = static_cast<int>(fl);
-  return __int_as_float(__float_as_int(p) + static_cast<int>(static_cast<unsigned>(e) << 23));
-}
-
 // Rotates this thread's query row with the table at `pos` and writes it,
 // bf16 and swizzled, into the 128x128 tile at `dst`.
 __device__ __forceinline__ void rotate_q_row(uint8_t *dst, int r, const __nv_bfloat16 *qrow,
