@@ -37,6 +37,10 @@ sys.path.insert(0, ROOT)
 from long_context_attention_bifocal_b200 import workloads as W  # noqa: E402
 
 METRIC = "bifocal prefill TFLOP/s & % bf16 peak; decode KV-read GB/s & % HBM"
+# DRAM bytes (read + write) of one full-size launch of the prefill kernel,
+# from ncu (dram__bytes_read.sum + dram__bytes_write.sum, one pass) on B200.
+# Must be re-measured (or set to None) whenever that kernel changes.
+PREFILL_TRAFFIC_BYTES = 79.507e9 + 1.067e9
 PREFILL_CFG = "qwen3_8b_L131072"
 DECODE_CFG = "qwen3_8b_decode_n131072"
 
@@ -315,7 +319,7 @@ def run_cuda(args):
             "peak_kind": f"bf16 dense, sustained, {src}",
             "unit": "TFLOP/s",
             "frac": round(achieved / bf16_sust, 4),
-            "traffic": None,
+            "traffic": PREFILL_TRAFFIC_BYTES,
         },
         "e2e": {
             "value": round(flops * e_steps * world / (e2e_ms / 1e3) / 1e12, 2),

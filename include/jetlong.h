@@ -151,7 +151,7 @@ jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped,
  *   Split partials go to a fixed array compiled into the library:
  *   1,048,576 floats (4 MiB), present on every GPU that loads the library until
  *   the process exits.  Sizes are accepted while
- *   B * Hq * n_splits * (D + 2) fits it (n_splits about 75 for B=1, Hq=32 at
+ *   B * Hq * n_splits * (D + 4) fits it (n_splits about 75 for B=1, Hq=32 at
  *   pos = 131071); larger sizes return JL_ERR_UNSUPPORTED with a message.
  *   The first call on each device looks up that array's device address (with
  *   that device current) and caches it; make that first call before any stream

@@ -294,7 +294,8 @@ __device__ __forceinline__ void decode_split_body(const SplitParams &p, const do
       acc += red[w][h][d] * f;
       lsum += red[w][h][kD + 1] * f;
     }
-    float *dst = p.ws + ((static_cast<int64_t>(b) * p.Hq + h0 + h) * p.n_chunks + c) * (kD + 2);
+    float *dst = p.ws + ((static_cast<int64_t>(b) * p.Hq + h0 + h) * p.n_chunks + c) *
+                            kDecodePartialFloats;
     dst[d] = acc;
     if (d == 0) {
       dst[kD] = mx;
@@ -316,24 +317,57 @@ __global__ void __launch_bounds__(kThreads)
   decode_split_body<NH, true>(p, th.t);
 }
 
-// One CTA per (batch, query head): merges the chunk partials.
-__global__ void __launch_bounds__(kD)
+// One CTA of 8 warps per (batch, query head) merges the chunk partials:
+// M = max_c m_c, weights 2^(m_c - M), O = sum_c w_c o_c / sum_c w_c l_c and
+// lse = (M + log2 sum_c w_c l_c) * ln 2.  Each warp accumulates every eighth
+// partial with 16-byte loads; the warps' sums are added in shared memory.
+constexpr int kCombineThreads = 256;
+__global__ void __launch_bounds__(kCombineThreads)
     bifocal_decode_combine_kernel(const float *__restrict__ ws, __nv_bfloat16 *__restrict__ out,
                                   float *__restrict__ lse, int n_chunks) {
+  constexpr int kW = kCombineThreads / 32;
+  __shared__ float part[kW][kD];
+  __shared__ float wmax[kW], wsum[kW];
   const int bh = blockIdx.x;
-  const int d = threadIdx.x;
-  const float *src = ws + static_cast<int64_t>(bh) * n_chunks * (kD + 2);
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const float *src = ws + static_cast<int64_t>(bh) * n_chunks * kDecodePartialFloats;
   float mx = -INFINITY;
-  for (int c = 0; c < n_chunks; ++c) mx = fmaxf(mx, src[c * (kD + 2) + kD]);
-  float acc = 0.f, lsum = 0.f;
-  for (int c = 0; c < n_chunks; ++c) {
-    const float mc = src[c * (kD + 2) + kD];
-    const float f = (mc == -INFINITY) ? 0.f : ex2(mc - mx);
-    acc += src[c * (kD + 2) + d] * f;
-    lsum += src[c * (kD + 2) + kD + 1] * f;
+  for (int c = t; c < n_chunks; c += kCombineThreads)
+    mx = fmaxf(mx, src[c * kDecodePartialFloats + kD]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) wmax[warp] = mx;
+  __syncthreads();
+  float M = wmax[0];
+#pragma unroll
+  for (int w = 1; w < kW; ++w) M = fmaxf(M, wmax[w]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lsum = 0.f;
+#pragma unroll 4
+  for (int c = warp; c < n_chunks; c += kW) {
+    const float *pc = src + static_cast<int64_t>(c) * kDecodePartialFloats;
+    const float mc = pc[kD];
+    const float f = (mc == -INFINITY) ? 0.f : ex2(mc - M);
+    const float4 v = *reinterpret_cast<const float4 *>(pc + 4 * lane);
+    acc.x = fmaf(f, v.x, acc.x);
+    acc.y = fmaf(f, v.y, acc.y);
+    acc.z = fmaf(f, v.z, acc.z);
+    acc.w = fmaf(f, v.w, acc.w);
+    lsum = fmaf(f, pc[kD + 1], lsum);
   }
-  out[static_cast<int64_t>(bh) * kD + d] = __float2bfloat16_rn(acc / lsum);
-  if (d == 0) lse[bh] = (mx + __log2f(lsum)) * 0.69314718055994530942f;
+  *reinterpret_cast<float4 *>(&part[warp][4 * lane]) = acc;
+  if (lane == 0) wsum[warp] = lsum;
+  __syncthreads();
+  if (t < kD) {
+    float o = 0.f, L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kW; ++w) {
+      o += part[w][t];
+      L += wsum[w];
+    }
+    out[static_cast<int64_t>(bh) * kD + t] = __float2bfloat16_rn(o / L);
+    if (t == 0) lse[bh] = (M + __log2f(L)) * 0.69314718055994530942f;
+  }
 }
 
 template <int NH>
@@ -342,7 +376,8 @@ cudaError_t launch_nh(const DecodeArgs &a, const SplitParams &sp, cudaStream_t s
   bifocal_decode_split_kernel<NH><<<grid, kThreads, 0, s>>>(sp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bifocal_decode_combine_kernel<<<a.B * a.Hq, kD, 0, s>>>(a.ws, a.out, a.lse, a.n_chunks);
+  bifocal_decode_combine_kernel<<<a.B * a.Hq, kCombineThreads, 0, s>>>(a.ws, a.out, a.lse,
+                                                                        a.n_chunks);
   return cudaGetLastError();
 }
 
@@ -353,7 +388,8 @@ cudaError_t launch_nh_selfangle(const DecodeArgs &a, const SplitParams &sp, cons
   bifocal_decode_split_selfangle_kernel<NH><<<grid, kThreads, 0, s>>>(sp, th);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bifocal_decode_combine_kernel<<<a.B * a.Hq, kD, 0, s>>>(a.ws, a.out, a.lse, a.n_chunks);
+  bifocal_decode_combine_kernel<<<a.B * a.Hq, kCombineThreads, 0, s>>>(a.ws, a.out, a.lse,
+                                                                        a.n_chunks);
   return cudaGetLastError();
 }
 
@@ -416,12 +452,13 @@ cudaError_t launch_decode_noalloc(const DecodeArgs &a_in, double rope_base, cuda
 }
 
 cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t s) {
-  bifocal_decode_combine_kernel<<<a.B * a.Hq, kD, 0, s>>>(a.ws, a.out, a.lse, a.n_chunks);
+  bifocal_decode_combine_kernel<<<a.B * a.Hq, kCombineThreads, 0, s>>>(a.ws, a.out, a.lse,
+                                                                        a.n_chunks);
   return cudaGetLastError();
 }
 
 size_t decode_ws_floats(int B, int Hq, int D, int n_chunks) {
-  return static_cast<size_t>(B) * Hq * n_chunks * (D + 2);
+  return static_cast<size_t>(B) * Hq * n_chunks * kDecodePartialFloats;
 }
 
 // Keys per chunk: enough chunks for about kTargetCtas CTAs, a multiple of 64,

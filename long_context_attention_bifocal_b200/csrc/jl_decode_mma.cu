@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = g + 8 * rr;
     if (row >= rows) continue;
     float *dst = p.ws + ((static_cast<int64_t>(b) * p.Hq + hk * p.group + row) * p.n_chunks + c) *
-                            (kD + 2);
+                            kDecodePartialFloats;
 #pragma unroll
     for (int nd = 0; nd < 16; ++nd) {
       dst[8 * nd + 2 * cq] = o[nd][2 * rr];

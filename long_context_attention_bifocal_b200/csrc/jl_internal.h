@@ -83,6 +83,10 @@ struct DecodeArgs {
   int n_far_chunks, n_chunks;
 };
 
+// One split partial in the decode workspace: o[128], m (log2 units), l, and
+// two floats of padding so every partial starts on a 16-byte boundary.
+constexpr int kDecodePartialFloats = 132;
+
 // Workspace floats for the given split layout.
 size_t decode_ws_floats(int B, int Hq, int D, int n_chunks);
 void decode_plan(int B, int Hq, int Hkv, int pos, int far_end, int *chunk,
