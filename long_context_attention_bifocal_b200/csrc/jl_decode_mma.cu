@@ -12,8 +12,9 @@
 // producer warp.  The producer streams 16-key blocks through a 3-stage ring in
 // shared memory with TMA: per block and head, K and V as two 64-column boxes
 // with the 128-byte swizzle (so ldmatrix reads are conflict-free), plus, for a
-// remote chunk, the 16 rows of the cos/sin table that the block's corrections
-// need (u = k - f(k) grows by at most one per key).  The tensor maps end at
+// remote chunk, the 16 rows of the cos/sin table (fp16 copy: the rotated key
+// is rounded to bf16 anyway, so the 2^-11 table rounding does not show) that
+// the block's corrections need (u = k - f(k) grows by at most one per key).  The tensor maps end at
 // key pos, so slots past pos read as zeros and are never touched.
 //
 // Consumer warp (kv head h, its group of g <= 16 query heads as the 16 rows of
@@ -53,7 +54,8 @@ constexpr int kProducerWarp = kMaxHeads;
 constexpr uint32_t kHalfTile = kBlock * 128;          // one 64-column box: 2 KiB
 constexpr uint32_t kHeadBytes = 2 * kHalfTile;        // K (or V) of one head: 4 KiB
 constexpr uint32_t kKBytes = kMaxHeads * kHeadBytes;  // 32 KiB
-constexpr uint32_t kTabBytes = kBlock * kHalf * 8;    // 16 table rows: 8 KiB
+constexpr uint32_t kTabBox = kBlock * 128;            // 16 rows x 32 fp16 pairs: 2 KiB
+constexpr uint32_t kTabBytes = 2 * kTabBox;           // pairs 0-31 | 32-63: 4 KiB
 constexpr uint32_t kStageBytes = 2 * kKBytes + kTabBytes;
 constexpr uint32_t kOffBar = kStages * kStageBytes;
 constexpr uint32_t kSmemAlloc = kOffBar + 64 + 1024;
@@ -169,11 +171,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (far) {
           const int u0 = k0 - k0 / p.G;
-          asm volatile(
-              "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-              " [%0], [%1, {%2, %3}], [%4];" ::"r"(st + 2 * kKBytes),
-              "l"(reinterpret_cast<uint64_t>(&tm_tab)), "r"(0), "r"(u0), "r"(bar(s))
-              : "memory");
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb)  // pairs 0-31, then 32-63 (64 halves each)
+            asm volatile(
+                "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+                " [%0], [%1, {%2, %3}], [%4];" ::"r"(st + 2 * kKBytes + hb * kTabBox),
+                "l"(reinterpret_cast<uint64_t>(&tm_tab)), "r"(64 * hb), "r"(u0), "r"(bar(s))
+                : "memory");
         }
         ++issued;
       }
@@ -275,13 +279,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         // this thread's key k0 + 8nt + g: rotate by -u theta_i
         const int kk = k0 + 8 * nt + g;
         const int urow = (kk - kk / p.G) - u0;  // 0..15
-        const float *trow = reinterpret_cast<const float *>(tab + urow * (kHalf * 8));
+        // row urow of the two swizzled boxes: pair i sits in box i / 32, line
+        // urow, 16-byte chunk ((i % 32) / 4) ^ (urow & 7), offset (i % 4) * 4
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int i0 = 16 * ks + 2 * cq + 8 * hh;  // pairs i0, i0+1
-            const float4 f = *reinterpret_cast<const float4 *>(trow + 2 * i0);
+            const int ib = i0 & 31;
+            const uint2 hf = *reinterpret_cast<const uint2 *>(
+                tab + (i0 >> 5) * kTabBox + urow * 128 + (((ib >> 2) ^ (urow & 7)) << 4) +
+                (ib & 3) * 4);
+            const float2 f01 = __half22float2(*reinterpret_cast<const __half2 *>(&hf.x));
+            const float2 f23 = __half22float2(*reinterpret_cast<const __half2 *>(&hf.y));
+            const float4 f = make_float4(f01.x, f01.y, f23.x, f23.y);
             const uint32_t lo = kb[ks][hh], hi = kb[ks + 4][hh];
             const float a0 = bf_lo(lo), a1 = bf_hi(lo), b0 = bf_lo(hi), b1 = bf_hi(hi);
             // (x1, x2) -> (x1 c + x2 s, x2 c - x1 s)
@@ -413,16 +424,16 @@ bool make_cache_map(CUtensorMap *m, const void *base, int B, int cap, int keys, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// cos/sin table [positions][64] float2 seen as fp32 [positions][128]
-bool make_table_map(CUtensorMap *m, const float2 *cs, int positions) {
+// fp16 cos/sin table [positions][64] half2 seen as fp16 [positions][128]
+bool make_table_map(CUtensorMap *m, const __half2 *cs16, int positions) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {2 * kHalf, static_cast<cuuint64_t>(positions)};
-  const cuuint64_t strides[1] = {2 * kHalf * 4};
-  const cuuint32_t box[2] = {2 * kHalf, kBlock};
+  const cuuint64_t strides[1] = {2 * kHalf * 2};
+  const cuuint32_t box[2] = {kHalf, kBlock};  // 32 pairs x 16 rows, 128-byte lines
   const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float2 *>(cs), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half2 *>(cs16), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -457,7 +468,7 @@ cudaError_t launch_decode_mma(const DecodeArgs &a, unsigned *status, cudaStream_
   CUtensorMap mk, mv, mt;
   if (!make_cache_map(&mk, a.kc, a.B, a.cap, a.pos + 1, a.Hkv) ||
       !make_cache_map(&mv, a.vc, a.B, a.cap, a.pos + 1, a.Hkv) ||
-      !make_table_map(&mt, a.table.cs, a.table.positions))
+      !make_table_map(&mt, a.table.cs16, a.table.positions))
     return cudaErrorInvalidValue;
   Params p;
   p.q = a.q;

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstddef>
 #include <cstdint>
 
@@ -20,8 +21,9 @@ enum : unsigned {
 // computed with fp64 sincos and rounded to fp32.
 struct RopeTable {
   const float2 *cs;
-  int positions;  // valid p in [0, positions)
-  int half;       // D / 2
+  const __half2 *cs16;  // the same angles as fp16 (cos, sin) pairs
+  int positions;        // valid p in [0, positions)
+  int half;             // D / 2
 };
 
 // Records a message for jl_last_error() and returns st.
@@ -36,7 +38,7 @@ jl_status prefill_scratch(size_t bytes, void **out);
 int sm_count();
 
 // ---- launchers (each returns the launch's cudaError_t) ----
-cudaError_t launch_rope_table(float2 *cs, int positions, int D, double base,
+cudaError_t launch_rope_table(float2 *cs, __half2 *cs16, int positions, int D, double base,
                               cudaStream_t s);
 
 // Rotated copies of the keys of a [B,L,Hkv,D] bf16 tensor:
