@@ -66,7 +66,18 @@ enum {
    * standard RoPE at its original positions (plain causal RoPE attention).
    * This is the overhead baseline; with G = 1 the bifocal call takes exactly
    * this path. */
-  JL_FLAG_NO_BIFOCAL = 1u << 0
+  JL_FLAG_NO_BIFOCAL = 1u << 0,
+  /* TEST ONLY (jl_bifocal_decode): exercises the kernels' bounded waits.  The
+   * decode kernel's TMA producer withholds its first arrival, so the consumer
+   * warps' wait on the first K/V block expires after about one second; they
+   * raise the device status word and every warp of the kernel returns without
+   * a copy in flight.  The call itself returns JL_OK (the launch succeeded),
+   * out and lse are invalid, and the next jl_check_device_status returns
+   * JL_ERR_TIMEOUT and clears the word, after which the library works as
+   * before.  Accepted only where the tensor-core decode kernel runs (D = 128,
+   * Hkv <= 8, Hq / Hkv <= 16), JL_ERR_UNSUPPORTED otherwise; every other
+   * entry point rejects it as an unknown flag. */
+  JL_FLAG_DEBUG_SKIP_ARRIVE = 1u << 31
 };
 
 /* G = max(1, ceil(L / w_pretrained)) (bittide summary §3.1).  Returns -1 when
@@ -125,7 +136,7 @@ size_t jl_bifocal_decode_workspace_size(int B, int Hq, int Hkv, int D, int pos);
  *   workspace: device memory of at least jl_bifocal_decode_workspace_size()
  *   bytes, 16-byte aligned (split-KV partial results).
  *   D == 128, 0 <= pos < cache_capacity, Hq % Hkv == 0.
- *   flags: JL_FLAG_NO_BIFOCAL.
+ *   flags: JL_FLAG_NO_BIFOCAL; JL_FLAG_DEBUG_SKIP_ARRIVE (tests only).
  */
 jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped,
                             const void *v_cache, int pos, int cache_capacity,

@@ -14,13 +14,14 @@ import os
 import torch
 
 __all__ = [
-    "NO_BIFOCAL", "JetLongError", "group_size", "bifocal_prefill",
+    "NO_BIFOCAL", "DEBUG_SKIP_ARRIVE", "JetLongError", "group_size", "bifocal_prefill",
     "prefill_workspace_size", "decode_workspace_size", "bifocal_decode",
     "bifocal_decode_noalloc",
     "check_device_status", "finalize", "library_path", "load",
 ]
 
 NO_BIFOCAL = 1 << 0  # JL_FLAG_NO_BIFOCAL
+DEBUG_SKIP_ARRIVE = 1 << 31  # JL_FLAG_DEBUG_SKIP_ARRIVE (tests of the bounded waits only)
 
 _BF16, _F32 = 0, 1
 _STATUS = {0: "JL_OK", 1: "JL_ERR_INVALID_ARG", 2: "JL_ERR_UNSUPPORTED",

@@ -31,7 +31,6 @@ struct DeviceState {
   bool init = false;
   int sms = 0;
   float2 *table = nullptr;
-  __half2 *table16 = nullptr;
   int table_positions = 0;
   int table_D = 0;
   double table_base = 0.0;
@@ -114,36 +113,25 @@ jl_status rope_table(int D, double base, int min_positions, cudaStream_t s, Rope
       cudaError_t e = cudaDeviceSynchronize();  // earlier kernels may still read it
       if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
       cudaFree(d->table);
-      cudaFree(d->table16);
       d->table = nullptr;
-      d->table16 = nullptr;
       d->table_positions = 0;
     }
     float2 *t = nullptr;
-    __half2 *t16 = nullptr;
     const size_t n = static_cast<size_t>(want) * (D / 2);
     cudaError_t e = cudaMalloc(&t, sizeof(float2) * n);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(rope table)");
-    e = cudaMalloc(&t16, sizeof(__half2) * n);
-    if (e != cudaSuccess) {
-      cudaFree(t);
-      return cuda_fail(e, "cudaMalloc(rope table fp16)");
-    }
-    e = launch_rope_table(t, t16, want, D, base, s);
+    e = launch_rope_table(t, want, D, base, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // usable from any stream after this
     if (e != cudaSuccess) {
       cudaFree(t);
-      cudaFree(t16);
       return cuda_fail(e, "rope table build");
     }
     d->table = t;
-    d->table16 = t16;
     d->table_positions = want;
     d->table_D = D;
     d->table_base = base;
   }
   out->cs = d->table;
-  out->cs16 = d->table16;
   out->positions = d->table_positions;
   out->half = D / 2;
   return JL_OK;
@@ -343,9 +331,13 @@ jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped, const 
   if (!aligned16(q_new) || !aligned16(k_cache_roped) || !aligned16(v_cache) ||
       !aligned16(out) || !aligned16(lse) || !aligned16(workspace))
     return fail(JL_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL)) != 0)
+  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL | JL_FLAG_DEBUG_SKIP_ARRIVE)) != 0)
     return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
   if (D != 128) return fail(JL_ERR_UNSUPPORTED, "decode supports head dim 128 (got %d)", D);
+  if ((flags & JL_FLAG_DEBUG_SKIP_ARRIVE) && !decode_mma_supported(Hq, Hkv, D))
+    return fail(JL_ERR_UNSUPPORTED,
+                "JL_FLAG_DEBUG_SKIP_ARRIVE needs the tensor-core decode kernel "
+                "(Hkv <= 8, Hq / Hkv <= 16)");
   if (cache_capacity < 1 || pos < 0 || pos >= cache_capacity)
     return fail(JL_ERR_INVALID_ARG, "need 0 <= pos (%d) < cache_capacity (%d)", pos,
                 cache_capacity);
@@ -375,6 +367,7 @@ jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped, const 
   const long long fe = static_cast<long long>(pos) + 1 - w_local;
   a.far_end = plain ? 0 : static_cast<int>(fe < 0 ? 0 : fe);
   a.scale = static_cast<float>(1.0 / std::sqrt(D));
+  a.debug_skip_arrival = (flags & JL_FLAG_DEBUG_SKIP_ARRIVE) != 0;
   st = rope_table(D, rope_base, pos + 1 < 64 ? 64 : pos + 1, s, &a.table);
   if (st != JL_OK) return st;
   cudaError_t e;
@@ -429,7 +422,7 @@ jl_status jl_bifocal_decode_noalloc(const void *q_new, const void *k_cache_roped
   const long long fe = static_cast<long long>(pos) + 1 - w_local;
   a.far_end = plain ? 0 : static_cast<int>(fe < 0 ? 0 : fe);
   a.scale = static_cast<float>(1.0 / std::sqrt(D));
-  a.table = RopeTable{nullptr, nullptr, 0, D / 2};
+  a.table = RopeTable{nullptr, 0, D / 2};
   decode_plan(B, Hq, Hkv, pos, a.far_end, &a.chunk, &a.n_far_chunks, &a.n_chunks);
   const size_t need = decode_ws_floats(B, Hq, D, a.n_chunks);
   if (need > kDecodeNoAllocFloats)
@@ -469,11 +462,9 @@ void jl_finalize(void) {
     if (cudaSetDevice(i) != cudaSuccess) continue;
     cudaDeviceSynchronize();
     if (d.table) cudaFree(d.table);
-    if (d.table16) cudaFree(d.table16);
     if (d.status) cudaFree(d.status);
     if (d.scratch) cudaFree(d.scratch);
     d.table = nullptr;
-    d.table16 = nullptr;
     d.status = nullptr;
     d.scratch = nullptr;
     d.table_positions = 0;

@@ -302,6 +302,9 @@ __device__ __forceinline__ void decode_split_body(const SplitParams &p, const do
       dst[kD + 1] = lsum;
     }
   }
+  // the combine kernel (a programmatic dependent) may be scheduled once every
+  // CTA got here; it waits for this grid's completion before reading
+  asm volatile("griddepcontrol.launch_dependents;");
 }
 
 template <int NH>
@@ -317,18 +320,24 @@ __global__ void __launch_bounds__(kThreads)
   decode_split_body<NH, true>(p, th.t);
 }
 
-// One CTA of 8 warps per (batch, query head) merges the chunk partials:
-// M = max_c m_c, weights 2^(m_c - M), O = sum_c w_c o_c / sum_c w_c l_c and
-// lse = (M + log2 sum_c w_c l_c) * ln 2.  Each warp accumulates every eighth
-// partial with 16-byte loads; the warps' sums are added in shared memory.
+// Merges the chunk partials: M = max_c m_c, weights 2^(m_c - M),
+// O = sum_c w_c o_c / sum_c w_c l_c, lse = (M + log2 sum_c w_c l_c) * ln 2.
+// One CTA of 8 warps per (batch, query head, 32-dim slice): every warp takes
+// every eighth chunk, one dim per lane (128-byte loads), and the warps' sums
+// are added in shared memory.  The kernel is launched as a programmatic
+// dependent of the split kernel: it may start while that kernel runs and
+// waits (griddepcontrol.wait) until the partials are complete and visible.
 constexpr int kCombineThreads = 256;
+constexpr int kCombineSlice = 32;
+constexpr int kCombineSlices = kD / kCombineSlice;
 __global__ void __launch_bounds__(kCombineThreads)
     bifocal_decode_combine_kernel(const float *__restrict__ ws, __nv_bfloat16 *__restrict__ out,
                                   float *__restrict__ lse, int n_chunks) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int kW = kCombineThreads / 32;
-  __shared__ float part[kW][kD];
+  __shared__ float part[kW][kCombineSlice];
   __shared__ float wmax[kW], wsum[kW];
-  const int bh = blockIdx.x;
+  const int bh = blockIdx.x / kCombineSlices, sl = blockIdx.x % kCombineSlices;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const float *src = ws + static_cast<int64_t>(bh) * n_chunks * kDecodePartialFloats;
   float mx = -INFINITY;
@@ -341,32 +350,27 @@ __global__ void __launch_bounds__(kCombineThreads)
   float M = wmax[0];
 #pragma unroll
   for (int w = 1; w < kW; ++w) M = fmaxf(M, wmax[w]);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float lsum = 0.f;
+  float acc = 0.f, lsum = 0.f;
 #pragma unroll 4
   for (int c = warp; c < n_chunks; c += kW) {
     const float *pc = src + static_cast<int64_t>(c) * kDecodePartialFloats;
     const float mc = pc[kD];
     const float f = (mc == -INFINITY) ? 0.f : ex2(mc - M);
-    const float4 v = *reinterpret_cast<const float4 *>(pc + 4 * lane);
-    acc.x = fmaf(f, v.x, acc.x);
-    acc.y = fmaf(f, v.y, acc.y);
-    acc.z = fmaf(f, v.z, acc.z);
-    acc.w = fmaf(f, v.w, acc.w);
+    acc = fmaf(f, pc[kCombineSlice * sl + lane], acc);
     lsum = fmaf(f, pc[kD + 1], lsum);
   }
-  *reinterpret_cast<float4 *>(&part[warp][4 * lane]) = acc;
+  part[warp][lane] = acc;
   if (lane == 0) wsum[warp] = lsum;
   __syncthreads();
-  if (t < kD) {
+  if (t < kCombineSlice) {
     float o = 0.f, L = 0.f;
 #pragma unroll
     for (int w = 0; w < kW; ++w) {
       o += part[w][t];
       L += wsum[w];
     }
-    out[static_cast<int64_t>(bh) * kD + t] = __float2bfloat16_rn(o / L);
-    if (t == 0) lse[bh] = (M + __log2f(L)) * 0.69314718055994530942f;
+    out[static_cast<int64_t>(bh) * kD + kCombineSlice * sl + t] = __float2bfloat16_rn(o / L);
+    if (sl == 0 && t == 0) lse[bh] = (M + __log2f(L)) * 0.69314718055994530942f;
   }
 }
 
@@ -376,9 +380,7 @@ cudaError_t launch_nh(const DecodeArgs &a, const SplitParams &sp, cudaStream_t s
   bifocal_decode_split_kernel<NH><<<grid, kThreads, 0, s>>>(sp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bifocal_decode_combine_kernel<<<a.B * a.Hq, kCombineThreads, 0, s>>>(a.ws, a.out, a.lse,
-                                                                        a.n_chunks);
-  return cudaGetLastError();
+  return launch_decode_combine(a, s);
 }
 
 template <int NH>
@@ -388,9 +390,7 @@ cudaError_t launch_nh_selfangle(const DecodeArgs &a, const SplitParams &sp, cons
   bifocal_decode_split_selfangle_kernel<NH><<<grid, kThreads, 0, s>>>(sp, th);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bifocal_decode_combine_kernel<<<a.B * a.Hq, kCombineThreads, 0, s>>>(a.ws, a.out, a.lse,
-                                                                        a.n_chunks);
-  return cudaGetLastError();
+  return launch_decode_combine(a, s);
 }
 
 // Split partials of the entry point that allocates nothing: a fixed array in
@@ -452,9 +452,18 @@ cudaError_t launch_decode_noalloc(const DecodeArgs &a_in, double rope_base, cuda
 }
 
 cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t s) {
-  bifocal_decode_combine_kernel<<<a.B * a.Hq, kCombineThreads, 0, s>>>(a.ws, a.out, a.lse,
-                                                                        a.n_chunks);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.B * a.Hq * kCombineSlices));
+  cfg.blockDim = dim3(kCombineThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, bifocal_decode_combine_kernel, static_cast<const float *>(a.ws),
+                            a.out, a.lse, a.n_chunks);
 }
 
 size_t decode_ws_floats(int B, int Hq, int D, int n_chunks) {

@@ -11,11 +11,15 @@
 // of one batch entry and ALL kv heads; one consumer warp per kv head, one
 // producer warp.  The producer streams 16-key blocks through a 3-stage ring in
 // shared memory with TMA: per block and head, K and V as two 64-column boxes
-// with the 128-byte swizzle (so ldmatrix reads are conflict-free), plus, for a
-// remote chunk, the 16 rows of the cos/sin table (fp16 copy: the rotated key
-// is rounded to bf16 anyway, so the 2^-11 table rounding does not show) that
-// the block's corrections need (u = k - f(k) grows by at most one per key).  The tensor maps end at
-// key pos, so slots past pos read as zeros and are never touched.
+// with the 128-byte swizzle (so ldmatrix reads are conflict-free).  For a
+// remote chunk the producer warp also writes the 16 rows of correction factors
+// (cos, sin)(u theta_i) that the block needs, u = k - f(k) growing by at most
+// one per key: row u0 + r is the complex product of the fp32 table row u0 (one
+// 512-byte read per block) and the step row r < 16 (held in registers), rounded
+// to fp16 (the rotated key is rounded to bf16 anyway, so the 2^-11 factor
+// rounding does not show).  So the corrections read no per-key data from HBM.
+// The tensor maps end at key pos, so slots past pos read as zeros and are never
+// touched.
 //
 // Consumer warp (kv head h, its group of g <= 16 query heads as the 16 rows of
 // an m16n8k16 bf16 MMA):
@@ -49,8 +53,9 @@ constexpr int kBlock = 16;            // keys per stage
 constexpr int kStages = 3;
 constexpr int kMaxHeads = 8;          // kv heads per CTA (one consumer warp each)
 constexpr int kMaxGroup = 16;         // query heads per kv head (MMA rows)
-constexpr int kThreads = (kMaxHeads + 1) * 32;
+constexpr int kThreads = (kMaxHeads + 2) * 32;
 constexpr int kProducerWarp = kMaxHeads;
+constexpr int kFactorWarp = kMaxHeads + 1;
 constexpr uint32_t kHalfTile = kBlock * 128;          // one 64-column box: 2 KiB
 constexpr uint32_t kHeadBytes = 2 * kHalfTile;        // K (or V) of one head: 4 KiB
 constexpr uint32_t kKBytes = kMaxHeads * kHeadBytes;  // 32 KiB
@@ -65,11 +70,12 @@ constexpr int kCtaTarget = 148;  // one wave of CTAs on a B200 per batch entry
 
 struct Params {
   const __nv_bfloat16 *q;
-  const float2 *cs;  // cos/sin table, for the query rotation
+  const float2 *cs;  // cos/sin table: query rotation, correction factors
   float *ws;
   unsigned *status;
   int Hq, Hkv, group, pos, G, far_end, chunk, n_far, n_chunks;
   float scale_log2;
+  int skip_first_arrival;  // test-only: withhold the first block (bounded-wait check)
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1,
@@ -111,8 +117,7 @@ __device__ __forceinline__ bool warp_wait_u(uint32_t bar, uint32_t parity,
 
 __global__ void __launch_bounds__(kThreads, 1)
     bifocal_decode_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
-                              const __grid_constant__ CUtensorMap tm_v,
-                              const __grid_constant__ CUtensorMap tm_tab, const Params p) {
+                              const __grid_constant__ CUtensorMap tm_v, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -131,12 +136,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nblk = (k_end - k_begin + kBlock - 1) / kBlock;
 
   auto bar = [&](int i) { return sb + kOffBar + 8u * static_cast<uint32_t>(i); };
-  // barriers: full[kStages], empty[kStages]; then abort flag
+  // barriers: full[kStages] (the producer's arrival with the TMA bytes, plus,
+  // in a remote chunk, the 32 lanes of the factor warp), empty[kStages] (one
+  // arrival per consumer warp); then the abort flag
   volatile int *abort_s = reinterpret_cast<volatile int *>(smem + kOffBar + 8 * 2 * kStages);
   volatile unsigned *abort_g = p.status;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(s), 1);
+      mbar_init(bar(s), far ? 33 : 1);
       mbar_init(bar(kStages + s), p.Hkv);
     }
     *abort_s = (*abort_g != 0u) ? 1 : 0;
@@ -149,10 +156,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      if (far) prefetch_tmap(&tm_tab);
-      const uint32_t bytes = static_cast<uint32_t>(p.Hkv) * 2 * kHeadBytes + (far ? kTabBytes : 0);
+      const uint32_t bytes = static_cast<uint32_t>(p.Hkv) * 2 * kHeadBytes;
       int issued = 0;
-      for (int blk = 0; blk < nblk; ++blk) {
+      // test-only: no block is loaded, so the consumers' first wait expires
+      for (int blk = p.skip_first_arrival ? nblk : 0; blk < nblk; ++blk) {
         const int s = blk % kStages;
         const uint32_t ph = (blk / kStages) & 1;
         if (!mbar_wait(bar(kStages + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
@@ -169,16 +176,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(st + kKBytes + h * kHeadBytes, &tm_v, bar(s), 0, h, k0, b);
           tma_load_4d(st + kKBytes + h * kHeadBytes + kHalfTile, &tm_v, bar(s), kHalf, h, k0, b);
         }
-        if (far) {
-          const int u0 = k0 - k0 / p.G;
-#pragma unroll
-          for (int hb = 0; hb < 2; ++hb)  // pairs 0-31, then 32-63 (64 halves each)
-            asm volatile(
-                "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-                " [%0], [%1, {%2, %3}], [%4];" ::"r"(st + 2 * kKBytes + hb * kTabBox),
-                "l"(reinterpret_cast<uint64_t>(&tm_tab)), "r"(64 * hb), "r"(u0), "r"(bar(s))
-                : "memory");
-        }
         ++issued;
       }
       // never leave with a copy in flight into this CTA's shared memory
@@ -187,6 +184,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (!mbar_try_wait(bar(d % kStages), (d / kStages) & 1))
           if (globaltimer_ns() - t0 > kTimeoutNs) break;
       }
+    }
+    return;
+  }
+  if (warp == kFactorWarp) {
+    if (!far) return;
+    // Correction factors of pairs i = lane (box 0) and i = lane + 32 (box 1).
+    // step[r] = (cos, sin)(r theta_i) for r < 16; the block base row u0 is read
+    // one block ahead so its latency overlaps the previous block.
+    float2 step[kBlock][2];
+#pragma unroll
+    for (int r = 0; r < kBlock; ++r) {
+      step[r][0] = p.cs[r * kHalf + lane];
+      step[r][1] = p.cs[r * kHalf + lane + 32];
+    }
+    int u0 = k_begin - k_begin / p.G;
+    float2 base0 = p.cs[static_cast<int64_t>(u0) * kHalf + lane];
+    float2 base1 = p.cs[static_cast<int64_t>(u0) * kHalf + lane + 32];
+    for (int blk = 0; blk < nblk; ++blk) {
+      const int s = blk % kStages;
+      const uint32_t ph = (blk / kStages) & 1;
+      if (!warp_wait_u(bar(kStages + s), ph ^ 1u, abort_s, abort_g)) {
+        if (lane == 0) {
+          *abort_s = 1;
+          atomicOr(p.status, kStatusTimeout);
+        }
+        break;
+      }
+      const float2 c0 = base0, c1 = base1;
+      if (blk + 1 < nblk) {
+        const int kn = k_begin + (blk + 1) * kBlock;
+        u0 = kn - kn / p.G;
+        base0 = p.cs[static_cast<int64_t>(u0) * kHalf + lane];
+        base1 = p.cs[static_cast<int64_t>(u0) * kHalf + lane + 32];
+      }
+      // line r of each box: pair (i % 32) in 16-byte chunk ((i % 32) / 4) ^ (r % 8)
+      uint8_t *tab = smem + s * kStageBytes + 2 * kKBytes;
+#pragma unroll
+      for (int r = 0; r < kBlock; ++r) {
+        const uint32_t off = r * 128 + ((((lane >> 2) ^ (r & 7)) << 4) | ((lane & 3) * 4));
+        const float2 a = step[r][0], d = step[r][1];
+        *reinterpret_cast<__half2 *>(tab + off) =
+            __floats2half2_rn(c0.x * a.x - c0.y * a.y, c0.y * a.x + c0.x * a.y);
+        *reinterpret_cast<__half2 *>(tab + kTabBox + off) =
+            __floats2half2_rn(c1.x * d.x - c1.y * d.y, c1.y * d.x + c1.x * d.y);
+      }
+      mbar_arrive(bar(s));  // release: this lane's factor writes
     }
     return;
   }
@@ -391,6 +434,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       dst[kD + 1] = l[rr];
     }
   }
+  // the combine kernel (a programmatic dependent) may be scheduled once every
+  // CTA got here; it waits for this grid's completion before reading
+  asm volatile("griddepcontrol.launch_dependents;");
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -424,20 +470,6 @@ bool make_cache_map(CUtensorMap *m, const void *base, int B, int cap, int keys, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp16 cos/sin table [positions][64] half2 seen as fp16 [positions][128]
-bool make_table_map(CUtensorMap *m, const __half2 *cs16, int positions) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {2 * kHalf, static_cast<cuuint64_t>(positions)};
-  const cuuint64_t strides[1] = {2 * kHalf * 2};
-  const cuuint32_t box[2] = {kHalf, kBlock};  // 32 pairs x 16 rows, 128-byte lines
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half2 *>(cs16), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool decode_mma_supported(int Hq, int Hkv, int D) {
@@ -465,10 +497,9 @@ cudaError_t launch_decode_mma(const DecodeArgs &a, unsigned *status, cudaStream_
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  CUtensorMap mk, mv, mt;
+  CUtensorMap mk, mv;
   if (!make_cache_map(&mk, a.kc, a.B, a.cap, a.pos + 1, a.Hkv) ||
-      !make_cache_map(&mv, a.vc, a.B, a.cap, a.pos + 1, a.Hkv) ||
-      !make_table_map(&mt, a.table.cs16, a.table.positions))
+      !make_cache_map(&mv, a.vc, a.B, a.cap, a.pos + 1, a.Hkv))
     return cudaErrorInvalidValue;
   Params p;
   p.q = a.q;
@@ -485,8 +516,9 @@ cudaError_t launch_decode_mma(const DecodeArgs &a, unsigned *status, cudaStream_
   p.n_far = a.n_far_chunks;
   p.n_chunks = a.n_chunks;
   p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.skip_first_arrival = a.debug_skip_arrival ? 1 : 0;
   dim3 grid(a.n_chunks, a.B);
-  bifocal_decode_mma_kernel<<<grid, kThreads, kSmemAlloc, s>>>(mk, mv, mt, p);
+  bifocal_decode_mma_kernel<<<grid, kThreads, kSmemAlloc, s>>>(mk, mv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_decode_combine(a, s);

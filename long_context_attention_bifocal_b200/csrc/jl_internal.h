@@ -21,9 +21,8 @@ enum : unsigned {
 // computed with fp64 sincos and rounded to fp32.
 struct RopeTable {
   const float2 *cs;
-  const __half2 *cs16;  // the same angles as fp16 (cos, sin) pairs
-  int positions;        // valid p in [0, positions)
-  int half;             // D / 2
+  int positions;  // valid p in [0, positions)
+  int half;       // D / 2
 };
 
 // Records a message for jl_last_error() and returns st.
@@ -38,8 +37,7 @@ jl_status prefill_scratch(size_t bytes, void **out);
 int sm_count();
 
 // ---- launchers (each returns the launch's cudaError_t) ----
-cudaError_t launch_rope_table(float2 *cs, __half2 *cs16, int positions, int D, double base,
-                              cudaStream_t s);
+cudaError_t launch_rope_table(float2 *cs, int positions, int D, double base, cudaStream_t s);
 
 // Rotated copies of the keys of a [B,L,Hkv,D] bf16 tensor:
 // kstd = R(l) k (if kstd), krem = R(floor(l/G)) k (if krem).
@@ -83,6 +81,7 @@ struct DecodeArgs {
   RopeTable table;
   int chunk;                // keys per split
   int n_far_chunks, n_chunks;
+  bool debug_skip_arrival = false;  // JL_FLAG_DEBUG_SKIP_ARRIVE (tensor-core kernel)
 };
 
 // One split partial in the decode workspace: o[128], m (log2 units), l, and

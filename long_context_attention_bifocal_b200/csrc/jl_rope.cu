@@ -16,9 +16,9 @@ struct Thetas {
 };
 
 // cs[p * half + i] = (cos(p theta_i), sin(p theta_i)): the angle and its sine
-// and cosine in fp64, rounded once to fp32 (cs) and once to fp16 (cs16).
-__global__ void rope_table_kernel(float2 *__restrict__ cs, __half2 *__restrict__ cs16,
-                                  int positions, int half, const Thetas th) {
+// and cosine in fp64, rounded once to fp32.
+__global__ void rope_table_kernel(float2 *__restrict__ cs, int positions, int half,
+                                  const Thetas th) {
   const int64_t n = static_cast<int64_t>(positions) * half;
   for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -27,7 +27,6 @@ __global__ void rope_table_kernel(float2 *__restrict__ cs, __half2 *__restrict__
     double s, c;
     sincos(static_cast<double>(p) * th.t[i], &s, &c);
     cs[idx] = make_float2(static_cast<float>(c), static_cast<float>(s));
-    cs16[idx] = __halves2half2(__double2half(c), __double2half(s));
   }
 }
 
@@ -93,8 +92,7 @@ __global__ void rotate_keys_kernel(const __nv_bfloat16 *__restrict__ k,
 
 }  // namespace
 
-cudaError_t launch_rope_table(float2 *cs, __half2 *cs16, int positions, int D, double base,
-                              cudaStream_t s) {
+cudaError_t launch_rope_table(float2 *cs, int positions, int D, double base, cudaStream_t s) {
   Thetas th;
   const int half = D / 2;
   for (int i = 0; i < half; ++i) th.t[i] = pow(base, -2.0 * i / D);
@@ -102,7 +100,7 @@ cudaError_t launch_rope_table(float2 *cs, __half2 *cs16, int positions, int D, d
   const int threads = 256;
   const int64_t blocks64 = (n + threads - 1) / threads;
   const int blocks = static_cast<int>(blocks64 < 65536 ? blocks64 : 65536);
-  rope_table_kernel<<<blocks, threads, 0, s>>>(cs, cs16, positions, half, th);
+  rope_table_kernel<<<blocks, threads, 0, s>>>(cs, positions, half, th);
   return cudaGetLastError();
 }
 

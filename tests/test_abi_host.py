@@ -77,6 +77,7 @@ INVALID, UNSUPPORTED = 1, 2
     (dict(q=None), INVALID),
     (dict(k=FAKE + 2), INVALID),          # misaligned
     (dict(flags=1 << 7), INVALID),
+    (dict(flags=1 << 31), INVALID),       # the decode-only test flag
     (dict(dtype=5), INVALID),
     (dict(ws=FAKE + 16, ws_bytes=1 << 30), INVALID),  # workspace not 256-aligned
     (dict(ws=FAKE, ws_bytes=10), INVALID),            # workspace too small
@@ -107,6 +108,7 @@ def _decode(lib, **kw):
     (dict(kc=FAKE + 4), INVALID),
     (dict(w_local=-3), INVALID),
     (dict(flags=2), INVALID),
+    (dict(Hq=34, Hkv=2, flags=1 << 31), UNSUPPORTED),  # group 17: no tensor-core kernel
 ])
 def test_decode_rejects(lib, kw, code):
     assert _decode(lib, **kw) == code
