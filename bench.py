@@ -239,8 +239,24 @@ def run_cuda(args):
         torch.cuda.synchronize()
         return sorted(a.elapsed_time(b) for a, b in es)[reps // 2]
 
-    dec_bif = avg_ms(lambda: decode(0), 50)
-    dec_plain = avg_ms(lambda: decode(jl.NO_BIFOCAL), 50)
+    def interleaved_ms(fa, fb, reps):
+        """Medians of fa and fb timed alternately (clock drift hits both)."""
+        ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        eb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        for (a0, a1), (b0, b1) in zip(ea, eb):
+            a0.record(stream)
+            fa()
+            a1.record(stream)
+            b0.record(stream)
+            fb()
+            b1.record(stream)
+        torch.cuda.synchronize()
+        med = lambda es: sorted(x.elapsed_time(y) for x, y in es)[reps // 2]  # noqa: E731
+        return med(ea), med(eb)
+
+    dec_bif, dec_plain = interleaved_ms(lambda: decode(0), lambda: decode(jl.NO_BIFOCAL), 100)
     pre_plain = avg_ms(lambda: prefill(jl.NO_BIFOCAL), max(1, min(3, args.steps)))
     pre_bif = avg_ms(lambda: prefill(0), max(1, min(3, args.steps)))
     jl.check_device_status()

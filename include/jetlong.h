@@ -75,7 +75,7 @@ enum {
    * out and lse are invalid, and the next jl_check_device_status returns
    * JL_ERR_TIMEOUT and clears the word, after which the library works as
    * before.  Accepted only where the tensor-core decode kernel runs (D = 128,
-   * Hkv <= 8, Hq / Hkv <= 16), JL_ERR_UNSUPPORTED otherwise; every other
+   * Hkv <= 8, Hq / Hkv <= 8), JL_ERR_UNSUPPORTED otherwise; every other
    * entry point rejects it as an unknown flag. */
   JL_FLAG_DEBUG_SKIP_ARRIVE = 1u << 31
 };

@@ -337,7 +337,7 @@ jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped, const 
   if ((flags & JL_FLAG_DEBUG_SKIP_ARRIVE) && !decode_mma_supported(Hq, Hkv, D))
     return fail(JL_ERR_UNSUPPORTED,
                 "JL_FLAG_DEBUG_SKIP_ARRIVE needs the tensor-core decode kernel "
-                "(Hkv <= 8, Hq / Hkv <= 16)");
+                "(Hkv <= 8, Hq / Hkv <= 8)");
   if (cache_capacity < 1 || pos < 0 || pos >= cache_capacity)
     return fail(JL_ERR_INVALID_ARG, "need 0 <= pos (%d) < cache_capacity (%d)", pos,
                 cache_capacity);

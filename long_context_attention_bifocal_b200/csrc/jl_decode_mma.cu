@@ -8,29 +8,32 @@
 // and scored against q_rem.  Softmax over all keys of the cache.
 //
 // B200 layout.  A CTA owns one chunk of keys (wholly remote or wholly local)
-// of one batch entry and ALL kv heads; one consumer warp per kv head, one
-// producer warp.  The producer streams 16-key blocks through a 3-stage ring in
-// shared memory with TMA: per block and head, K and V as two 64-column boxes
-// with the 128-byte swizzle (so ldmatrix reads are conflict-free).  For a
-// remote chunk the producer warp also writes the 16 rows of correction factors
-// (cos, sin)(u theta_i) that the block needs, u = k - f(k) growing by at most
-// one per key: row u0 + r is the complex product of the fp32 table row u0 (one
-// 512-byte read per block) and the step row r < 16 (held in registers), rounded
-// to fp16 (the rotated key is rounded to bf16 anyway, so the 2^-11 factor
-// rounding does not show).  So the corrections read no per-key data from HBM.
-// The tensor maps end at key pos, so slots past pos read as zeros and are never
-// touched.
+// of one batch entry and ALL kv heads: one consumer warp per kv head, a TMA
+// producer warp and, in a remote chunk, a factor warp.  The producer streams
+// 16-key blocks through a 3-stage ring in shared memory: per block and head, K
+// and V as two 64-column boxes with the 128-byte swizzle (so ldmatrix reads
+// are conflict-free), one box per producer lane.  The tensor maps end at key pos, so slots past pos read
+// as zeros and are never touched.  The factor warp writes, per block, the 16
+// rows of correction factors (cos, sin)(u theta_i) the block needs (u = k -
+// f(k) grows by at most one per key): row u0 + r is the complex product of the
+// fp32 table row u0 (one 512-byte read per block) and the step row r < 16
+// (held in registers), rounded to bf16, so the corrections read no per-key
+// data from HBM.
 //
-// Consumer warp (kv head h, its group of g <= 16 query heads as the 16 rows of
-// an m16n8k16 bf16 MMA):
-//   S^T[head][key] = Q . K^T      8 k-steps x 2 key tiles, Q fragments held
-//                                 in registers (pre-rotated, pre-scaled)
-//   K fragments (ldmatrix) of a remote key are rotated by -u*theta_i in fp32:
-//   pair (i, i+64) lives in k-steps ks and ks+4 of the same thread, the factor
-//   (cos, sin)(u theta_i) is read from the staged table row.
-//   online softmax per query row (fp32, base 2, rescale only when the running
-//   max grows by more than 2^8), P packed straight from the S accumulators
-//   into the A fragments of O += P . V (V fragments by ldmatrix.trans).
+// Consumer warp (kv head h, its group of <= 8 query heads): m16n8k16 bf16 MMAs
+// with the block's 16 keys as rows and the query heads as columns, so that no
+// MMA row is padding:
+//   S = K . Q^T          8 k-steps, Q^T fragments held in registers
+//                        (pre-rotated, pre-scaled by log2(e)/sqrt(D))
+//   K fragments (ldmatrix) of a remote key are rotated by -u theta_i with
+//   packed bf16x2 multiply-adds: pair (i, i+64) lies in k-steps ks and ks+4 of
+//   the same thread.  (fp32 arithmetic here costs about 11 instructions per
+//   two pairs instead of 5 and, on a B200, 8% of decode time at n = 131072;
+//   the rotated key is rounded to bf16 for the MMA either way, and the extra
+//   roundings leave the error against the fp64 reference within 1.5x.)
+//   online softmax per head column (fp32, base 2, rescale only when the
+//   running max grows by more than 2^8); P is transposed into the B fragments
+//   of O^T += V^T . P^T with movmatrix (V^T fragments by ldmatrix.trans).
 // Each warp writes (o, m, l) of its heads for the chunk; the combine kernel of
 // jl_decode.cu merges the chunks.  Waits are bounded; a timeout raises the
 // device status word and the kernel returns.
@@ -52,15 +55,15 @@ constexpr int kHalf = 64;
 constexpr int kBlock = 16;            // keys per stage
 constexpr int kStages = 3;
 constexpr int kMaxHeads = 8;          // kv heads per CTA (one consumer warp each)
-constexpr int kMaxGroup = 16;         // query heads per kv head (MMA rows)
+constexpr int kMaxGroup = 8;          // query heads per kv head (MMA columns)
 constexpr int kThreads = (kMaxHeads + 2) * 32;
 constexpr int kProducerWarp = kMaxHeads;
 constexpr int kFactorWarp = kMaxHeads + 1;
 constexpr uint32_t kHalfTile = kBlock * 128;          // one 64-column box: 2 KiB
 constexpr uint32_t kHeadBytes = 2 * kHalfTile;        // K (or V) of one head: 4 KiB
 constexpr uint32_t kKBytes = kMaxHeads * kHeadBytes;  // 32 KiB
-constexpr uint32_t kTabBox = kBlock * 128;            // 16 rows x 32 fp16 pairs: 2 KiB
-constexpr uint32_t kTabBytes = 2 * kTabBox;           // pairs 0-31 | 32-63: 4 KiB
+constexpr uint32_t kTabRow = 32 * 8;                  // 32 x (cos, cos | sin, sin) bf16x2
+constexpr uint32_t kTabBytes = kBlock * kTabRow;      // 16 rows: 4 KiB
 constexpr uint32_t kStageBytes = 2 * kKBytes + kTabBytes;
 constexpr uint32_t kOffBar = kStages * kStageBytes;
 constexpr uint32_t kSmemAlloc = kOffBar + 64 + 1024;
@@ -75,6 +78,7 @@ struct Params {
   unsigned *status;
   int Hq, Hkv, group, pos, G, far_end, chunk, n_far, n_chunks;
   float scale_log2;
+  unsigned long long g_magic;  // ceil(2^64 / G): floor(k / G) = umulhi(k, g_magic), G >= 2
   int skip_first_arrival;  // test-only: withhold the first block (bounded-wait check)
 };
 
@@ -99,8 +103,35 @@ __device__ __forceinline__ void mma16816(float *d, uint32_t a0, uint32_t a1, uin
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+// floor(k / G) for 0 <= k < 2^31 and G >= 2, with magic = ceil(2^64 / G):
+// k * magic / 2^64 exceeds k / G by less than k * G / (G 2^64) < 1 / G, so the
+// floor is exact.
+__device__ __forceinline__ int div_g(int k, unsigned long long magic) {
+  return static_cast<int>(__umul64hi(static_cast<unsigned long long>(k), magic));
+}
+
+// 8x8 b16 matrix transpose across the warp
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// Rotates two pairs: lo holds x1 of pairs (j, j+1) and hi their x2, as
+// bf16x2; c2 = (c_j, c_j+1), s2 = (s_j, s_j+1) as bf16x2.
+// (x1, x2) -> (x1 c + x2 s, x2 c - x1 s): one product rounded to bf16, then a
+// fused multiply-add rounded once.
+__device__ __forceinline__ void rotate_pairs_bf(uint32_t &lo, uint32_t &hi, uint32_t c2,
+                                                uint32_t s2) {
+  uint32_t t, u, nl, nh;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(t) : "r"(hi), "r"(s2));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(nl) : "r"(lo), "r"(c2), "r"(t));
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(u) : "r"(lo), "r"(s2));
+  asm("neg.bf16x2 %0, %0;" : "+r"(u));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(nh) : "r"(hi), "r"(c2), "r"(u));
+  lo = nl;
+  hi = nh;
+}
 
 // byte offset of 16-byte chunk `ch` (0..15 over the 128 dims) of key row `row`
 // in a head's [2 halves][16 keys][128 B] swizzled tile
@@ -153,32 +184,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (*abort_s) return;
 
   if (warp == kProducerWarp) {
+    // One box per lane: lane j loads (head j / 4) K or V (j & 2), dims
+    // 0-63 or 64-127 (j & 1).  Issued by 32 lanes at once, the 32 copies of a
+    // block leave in a few cycles; a single issuing thread would take ~80
+    // cycles per copy and bound the kernel.
     if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      const uint32_t bytes = static_cast<uint32_t>(p.Hkv) * 2 * kHeadBytes;
-      int issued = 0;
-      // test-only: no block is loaded, so the consumers' first wait expires
-      for (int blk = p.skip_first_arrival ? nblk : 0; blk < nblk; ++blk) {
-        const int s = blk % kStages;
-        const uint32_t ph = (blk / kStages) & 1;
-        if (!mbar_wait(bar(kStages + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
+    }
+    const int h = lane >> 2;
+    const bool is_v = (lane & 2) != 0;
+    const int x = (lane & 1) * kHalf;
+    const CUtensorMap *map = is_v ? &tm_v : &tm_k;
+    const uint32_t dst_off =
+        (is_v ? kKBytes : 0u) + h * kHeadBytes + ((lane & 1) ? kHalfTile : 0u);
+    const uint32_t bytes = static_cast<uint32_t>(p.Hkv) * 2 * kHeadBytes;
+    int issued = 0;
+    // test-only: no block is loaded, so the consumers' first wait expires
+    for (int blk = p.skip_first_arrival ? nblk : 0; blk < nblk; ++blk) {
+      const int s = blk % kStages;
+      const uint32_t ph = (blk / kStages) & 1;
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait(bar(kStages + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs);
+        if (ok) mbar_arrive_expect_tx(bar(s), bytes);
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) {
           *abort_s = 1;
           atomicOr(p.status, kStatusTimeout);
-          break;
         }
-        const int k0 = k_begin + blk * kBlock;
-        const uint32_t st = sb + s * kStageBytes;
-        mbar_arrive_expect_tx(bar(s), bytes);
-        for (int h = 0; h < p.Hkv; ++h) {
-          tma_load_4d(st + h * kHeadBytes, &tm_k, bar(s), 0, h, k0, b);
-          tma_load_4d(st + h * kHeadBytes + kHalfTile, &tm_k, bar(s), kHalf, h, k0, b);
-          tma_load_4d(st + kKBytes + h * kHeadBytes, &tm_v, bar(s), 0, h, k0, b);
-          tma_load_4d(st + kKBytes + h * kHeadBytes + kHalfTile, &tm_v, bar(s), kHalf, h, k0, b);
-        }
-        ++issued;
+        break;
       }
-      // never leave with a copy in flight into this CTA's shared memory
+      if (h < p.Hkv)
+        tma_load_4d(sb + s * kStageBytes + dst_off, map, bar(s), x, h,
+                    k_begin + blk * kBlock, b);
+      ++issued;
+    }
+    // never leave with a copy in flight into this CTA's shared memory
+    if (lane == 0) {
       for (int d = (issued > kStages ? issued - kStages : 0); d < issued; ++d) {
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(bar(d % kStages), (d / kStages) & 1))
@@ -189,18 +233,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == kFactorWarp) {
     if (!far) return;
-    // Correction factors of pairs i = lane (box 0) and i = lane + 32 (box 1).
-    // step[r] = (cos, sin)(r theta_i) for r < 16; the block base row u0 is read
-    // one block ahead so its latency overlaps the previous block.
-    float2 step[kBlock][2];
+    // Correction factors of pairs 2 lane and 2 lane + 1: step[r] = (cos, sin)
+    // (r theta) of both, r < 16; the block's base row u0 is read one block
+    // ahead so its latency overlaps the previous block.
+    const float4 *cs4 = reinterpret_cast<const float4 *>(p.cs);
+    float4 step[kBlock];
 #pragma unroll
-    for (int r = 0; r < kBlock; ++r) {
-      step[r][0] = p.cs[r * kHalf + lane];
-      step[r][1] = p.cs[r * kHalf + lane + 32];
-    }
-    int u0 = k_begin - k_begin / p.G;
-    float2 base0 = p.cs[static_cast<int64_t>(u0) * kHalf + lane];
-    float2 base1 = p.cs[static_cast<int64_t>(u0) * kHalf + lane + 32];
+    for (int r = 0; r < kBlock; ++r) step[r] = cs4[r * (kHalf / 2) + lane];
+    int u0 = k_begin - div_g(k_begin, p.g_magic);
+    float4 base = cs4[static_cast<int64_t>(u0) * (kHalf / 2) + lane];
     for (int blk = 0; blk < nblk; ++blk) {
       const int s = blk % kStages;
       const uint32_t ph = (blk / kStages) & 1;
@@ -211,23 +252,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         break;
       }
-      const float2 c0 = base0, c1 = base1;
+      const float4 cb = base;
       if (blk + 1 < nblk) {
         const int kn = k_begin + (blk + 1) * kBlock;
-        u0 = kn - kn / p.G;
-        base0 = p.cs[static_cast<int64_t>(u0) * kHalf + lane];
-        base1 = p.cs[static_cast<int64_t>(u0) * kHalf + lane + 32];
+        u0 = kn - div_g(kn, p.g_magic);
+        base = cs4[static_cast<int64_t>(u0) * (kHalf / 2) + lane];
       }
-      // line r of each box: pair (i % 32) in 16-byte chunk ((i % 32) / 4) ^ (r % 8)
+      // row r, 8-byte word lane ^ (4 (r % 4)): (c0, c1 | s0, s1) as bf16x2
+      // of pairs 2 lane, 2 lane + 1 at angle (u0 + r) theta
       uint8_t *tab = smem + s * kStageBytes + 2 * kKBytes;
 #pragma unroll
       for (int r = 0; r < kBlock; ++r) {
-        const uint32_t off = r * 128 + ((((lane >> 2) ^ (r & 7)) << 4) | ((lane & 3) * 4));
-        const float2 a = step[r][0], d = step[r][1];
-        *reinterpret_cast<__half2 *>(tab + off) =
-            __floats2half2_rn(c0.x * a.x - c0.y * a.y, c0.y * a.x + c0.x * a.y);
-        *reinterpret_cast<__half2 *>(tab + kTabBox + off) =
-            __floats2half2_rn(c1.x * d.x - c1.y * d.y, c1.y * d.x + c1.x * d.y);
+        const float4 a = step[r];
+        const uint2 v = make_uint2(pack_bf16x2(cb.x * a.x - cb.y * a.y, cb.z * a.z - cb.w * a.w),
+                                   pack_bf16x2(cb.y * a.x + cb.x * a.y, cb.w * a.z + cb.z * a.w));
+        *reinterpret_cast<uint2 *>(tab + r * kTabRow + ((lane ^ ((r & 3) << 2)) << 3)) = v;
       }
       mbar_arrive(bar(s));  // release: this lane's factor writes
     }
@@ -236,58 +275,66 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= p.Hkv) return;
 
   // ------------------------------------------------------------ consumers --
+  // Warp = kv head hk.  m16n8k16 MMAs with the 16 keys of a block as the rows
+  // and the group's query heads (<= 8) as the columns:
+  //   S[key][head] = K . Q^T        A = K (ldmatrix), B = Q^T held in registers
+  //   O^T[dim][head] += V^T . P^T   A = V^T (ldmatrix.trans), B = P^T
+  // P moves from the accumulator layout of S to the B layout of P^T with two
+  // 8x8 transposes (movmatrix).
   const int hk = warp;
   const int g = lane >> 2, cq = lane & 3;  // MMA fragment coordinates
-  const int rows = p.group;                // real query rows of the MMA
-  // Q fragments: a[ks][0..3] = rows (g, g+8) x dims 16ks + 2cq + {0,1} / +8
-  uint32_t qa[8][4];
+  const int heads = p.group;               // real columns of the MMAs
+  // Q^T fragments: qb[ks][hh] = head g, dims 16ks + 2cq + 8hh + {0,1}
+  uint32_t qb[8][2];
   {
     const int udq = p.pos - p.pos / p.G;
+    const bool real = g < heads;
+    const __nv_bfloat16 *src =
+        p.q + (static_cast<int64_t>(b) * p.Hq + hk * p.group + (real ? g : 0)) * kD;
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      const int row = g + 8 * rr;
-      const bool real = row < rows;
-      const __nv_bfloat16 *src =
-          p.q + (static_cast<int64_t>(b) * p.Hq + hk * p.group + (real ? row : 0)) * kD;
+    for (int ks = 0; ks < 4; ++ks) {
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
+      for (int hh = 0; hh < 2; ++hh) {
+        const int d0 = 16 * ks + 2 * cq + 8 * hh;
+        float y1[2], y2[2];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {  // dims 16ks + 2cq + 8hh + {0,1}
-          const int d0 = 16 * ks + 2 * cq + 8 * hh;
-          float y1[2], y2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int i = d0 + e;  // rotation pair (i, i + 64)
-            const float x1 = real ? __bfloat162float(src[i]) : 0.f;
-            const float x2 = real ? __bfloat162float(src[i + kHalf]) : 0.f;
-            const float2 a = p.cs[static_cast<int64_t>(p.pos) * kHalf + i];
-            float z1 = x1 * a.x - x2 * a.y;
-            float z2 = x1 * a.y + x2 * a.x;
-            if (far) {  // by dq = -udq
-              const float2 r = p.cs[static_cast<int64_t>(udq) * kHalf + i];
-              const float w1 = z1 * r.x + z2 * r.y;
-              const float w2 = z2 * r.x - z1 * r.y;
-              z1 = w1;
-              z2 = w2;
-            }
-            y1[e] = z1 * p.scale_log2;
-            y2[e] = z2 * p.scale_log2;
+        for (int e = 0; e < 2; ++e) {
+          const int i = d0 + e;  // rotation pair (i, i + 64)
+          const float x1 = real ? __bfloat162float(src[i]) : 0.f;
+          const float x2 = real ? __bfloat162float(src[i + kHalf]) : 0.f;
+          const float2 a = p.cs[static_cast<int64_t>(p.pos) * kHalf + i];
+          float z1 = x1 * a.x - x2 * a.y;
+          float z2 = x1 * a.y + x2 * a.x;
+          if (far) {  // by dq = -udq
+            const float2 r = p.cs[static_cast<int64_t>(udq) * kHalf + i];
+            const float w1 = z1 * r.x + z2 * r.y;
+            const float w2 = z2 * r.x - z1 * r.y;
+            z1 = w1;
+            z2 = w2;
           }
-          // A fragment regs: [0] row g lo cols, [1] row g+8 lo, [2] row g hi, [3] row g+8 hi
-          qa[ks][2 * hh + rr] = pack_bf16x2(y1[0], y1[1]);
-          qa[ks + 4][2 * hh + rr] = pack_bf16x2(y2[0], y2[1]);
+          y1[e] = z1 * p.scale_log2;
+          y2[e] = z2 * p.scale_log2;
         }
+        qb[ks][hh] = pack_bf16x2(y1[0], y1[1]);
+        qb[ks + 4][hh] = pack_bf16x2(y2[0], y2[1]);
       }
     }
   }
 
-  float o[16][4];
+  // O^T accumulators of dim tile mt: [0] (dim 16mt+g, head 2cq), [1] (head
+  // 2cq+1), [2] (dim 16mt+g+8, head 2cq), [3] (head 2cq+1)
+  float o[8][4];
 #pragma unroll
-  for (int nd = 0; nd < 16; ++nd)
+  for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[nd][e] = 0.f;
-  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    for (int e = 0; e < 4; ++e) o[mt][e] = 0.f;
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};  // heads 2cq, 2cq+1
   bool ok = true;
+  // ldmatrix row supplied by this lane: K (A, matrices keys 0-7 | 8-15 x
+  // chunk 2ks | 2ks+1) and V^T (A by .trans, matrices chunk 2mt | 2mt+1 x keys
+  // 0-7 | 8-15)
+  const int krow = (lane & 7) + 8 * ((lane >> 3) & 1);
+  const int vrow = (lane & 7) + 8 * (lane >> 4);
 
   for (int blk = 0; blk < nblk; ++blk) {
     const int s = blk % kStages;
@@ -299,139 +346,129 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int k0 = k_begin + blk * kBlock;
     const uint32_t kt = sb + s * kStageBytes + hk * kHeadBytes;
     const uint32_t vt = kt + kKBytes;
-    const uint8_t *tab = smem + s * kStageBytes + 2 * kKBytes;
-    const int u0 = k0 - k0 / p.G;
 
-    // S^T = Q K^T for key tiles nt = 0, 1 (keys k0 + 8nt + [0, 8))
-    float sacc[2][4];
+    // K fragments kf[ks]: [0] key g, [1] key g+8 (dims 16ks + 2cq + {0,1}),
+    // [2], [3] the same keys at dims + 8
+    uint32_t kf[8][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+    for (int ks = 0; ks < 8; ++ks)
+      ldsm_x4(kt + tile_off(krow, 2 * ks + (lane >> 4)), kf[ks][0], kf[ks][1], kf[ks][2],
+              kf[ks][3]);
+    if (far) {
+      // a remote key is rotated by -u theta_i, u = k - f(k): pair (i, i+64)
+      // lies in k-steps ks and ks+4 of this thread; row u - u0 of the staged
+      // factors holds (cos, sin) of pairs (2pp, 2pp+1) in 8-byte word
+      // pp ^ (4 (row % 4)) as (c0, c1 | s0, s1), bf16x2 (conflict-free: the
+      // keys of a half-warp fall on at most 4 consecutive rows)
+      const uint8_t *tab = smem + s * kStageBytes + 2 * kKBytes;
+      const int u0 = k0 - div_g(k0, p.g_magic);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-      // K fragments: kb[ks][0..1]; ldmatrix row = key 8nt + (lane & 7),
-      // matrix (lane >> 3) -> 16-byte chunk 2*ks2 + (lane >> 3)
-      uint32_t kb[8][2];
-      const int krow = 8 * nt + (lane & 7);
-#pragma unroll
-      for (int ks2 = 0; ks2 < 8; ks2 += 2) {
-        const int ch = 2 * ks2 + (lane >> 3);
-        ldsm_x4(kt + tile_off(krow, ch), kb[ks2][0], kb[ks2][1], kb[ks2 + 1][0],
-                kb[ks2 + 1][1]);
-      }
-      if (far) {
-        // this thread's key k0 + 8nt + g: rotate by -u theta_i
-        const int kk = k0 + 8 * nt + g;
-        const int urow = (kk - kk / p.G) - u0;  // 0..15
-        // row urow of the two swizzled boxes: pair i sits in box i / 32, line
-        // urow, 16-byte chunk ((i % 32) / 4) ^ (urow & 7), offset (i % 4) * 4
+      for (int r = 0; r < 2; ++r) {
+        const int kk = k0 + g + 8 * r;
+        const int urow = (kk - div_g(kk, p.g_magic)) - u0;  // 0..15
+        const uint8_t *trow = tab + urow * kTabRow;
+        const int sw = (urow & 3) << 2;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
-            const int i0 = 16 * ks + 2 * cq + 8 * hh;  // pairs i0, i0+1
-            const int ib = i0 & 31;
-            const uint2 hf = *reinterpret_cast<const uint2 *>(
-                tab + (i0 >> 5) * kTabBox + urow * 128 + (((ib >> 2) ^ (urow & 7)) << 4) +
-                (ib & 3) * 4);
-            const float2 f01 = __half22float2(*reinterpret_cast<const __half2 *>(&hf.x));
-            const float2 f23 = __half22float2(*reinterpret_cast<const __half2 *>(&hf.y));
-            const float4 f = make_float4(f01.x, f01.y, f23.x, f23.y);
-            const uint32_t lo = kb[ks][hh], hi = kb[ks + 4][hh];
-            const float a0 = bf_lo(lo), a1 = bf_hi(lo), b0 = bf_lo(hi), b1 = bf_hi(hi);
-            // (x1, x2) -> (x1 c + x2 s, x2 c - x1 s)
-            kb[ks][hh] = pack_bf16x2(a0 * f.x + b0 * f.y, a1 * f.z + b1 * f.w);
-            kb[ks + 4][hh] = pack_bf16x2(b0 * f.x - a0 * f.y, b1 * f.z - a1 * f.w);
+            const int pp = 8 * ks + cq + 4 * hh;  // pairs 2pp, 2pp + 1
+            const uint2 f = *reinterpret_cast<const uint2 *>(trow + ((pp ^ sw) << 3));
+            rotate_pairs_bf(kf[ks][2 * hh + r], kf[ks + 4][2 * hh + r], f.x, f.y);
           }
         }
       }
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        mma16816(sacc[nt], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], kb[ks][0], kb[ks][1]);
     }
-    // sacc[nt][0..1]: row g, keys 8nt + 2cq + {0,1}; [2..3]: row g+8
-    if (k0 < k_begin || k0 + kBlock > k_end) {
+    // V^T fragments of the 8 dim tiles, then the stage goes back to the
+    // producer: the rest of the block works from registers
+    uint32_t vf[8][4];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+    for (int mt = 0; mt < 8; ++mt)
+      ldsm_x4_t(vt + tile_off(vrow, 2 * mt + ((lane >> 3) & 1)), vf[mt][0], vf[mt][1], vf[mt][2],
+                vf[mt][3]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(kStages + s));
+    // S = K . Q^T, two accumulation chains
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int kk = k0 + 8 * nt + 2 * cq + (e & 1);
-          if (kk >= k_end) sacc[nt][e] = -INFINITY;
-        }
+    for (int ks = 0; ks < 8; ks += 2) {
+      mma16816(sa, kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3], qb[ks][0], qb[ks][1]);
+      mma16816(sc, kf[ks + 1][0], kf[ks + 1][1], kf[ks + 1][2], kf[ks + 1][3], qb[ks + 1][0],
+               qb[ks + 1][1]);
+    }
+    // sv[0..1]: key g, heads 2cq, 2cq+1; sv[2..3]: key g+8
+    float sv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sv[e] = sa[e] + sc[e];
+    if (k0 + kBlock > k_end) {
+      if (k0 + g >= k_end) sv[0] = sv[1] = -INFINITY;
+      if (k0 + g + 8 >= k_end) sv[2] = sv[3] = -INFINITY;
     }
     float alpha[2];
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      float mx = fmaxf(fmaxf(sacc[0][2 * rr], sacc[0][2 * rr + 1]),
-                       fmaxf(sacc[1][2 * rr], sacc[1][2 * rr + 1]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      alpha[rr] = 1.f;
-      if (mx > m[rr] + 8.f) {
-        alpha[rr] = ex2_approx(m[rr] - mx);
-        m[rr] = mx;
+    for (int e = 0; e < 2; ++e) {
+      float mx = fmaxf(sv[e], sv[2 + e]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      alpha[e] = 1.f;
+      if (mx > m[e] + 8.f) {  // lazy rescale: only when the max grows by > 2^8
+        alpha[e] = ex2_approx(m[e] - mx);
+        m[e] = mx;
       }
     }
     if (alpha[0] != 1.f || alpha[1] != 1.f) {
 #pragma unroll
-      for (int nd = 0; nd < 16; ++nd) {
-        o[nd][0] *= alpha[0];
-        o[nd][1] *= alpha[0];
-        o[nd][2] *= alpha[1];
-        o[nd][3] *= alpha[1];
+      for (int mt = 0; mt < 8; ++mt) {
+        o[mt][0] *= alpha[0];
+        o[mt][1] *= alpha[1];
+        o[mt][2] *= alpha[0];
+        o[mt][3] *= alpha[1];
       }
       l[0] *= alpha[0];
       l[1] *= alpha[1];
     }
-    uint32_t pa[4];
+    float pv[4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const float mu = (m[rr] == -INFINITY) ? 0.f : m[rr];
-        const float p0 = ex2_approx(sacc[nt][2 * rr] - mu);
-        const float p1 = ex2_approx(sacc[nt][2 * rr + 1] - mu);
-        l[rr] += p0 + p1;
-        pa[2 * nt + rr] = pack_bf16x2(p0, p1);
-      }
+    for (int e = 0; e < 4; ++e) {
+      const float mu = (m[e & 1] == -INFINITY) ? 0.f : m[e & 1];
+      pv[e] = ex2_approx(sv[e] - mu);
     }
-    // O += P V over 16 dim tiles; V fragments by ldmatrix.trans:
-    // matrix (lane >> 3): keys 8*((lane>>3)&1) + (lane&7), dim chunk nd + (lane >> 4)
-    const int vrow = 8 * ((lane >> 3) & 1) + (lane & 7);
+    l[0] += pv[0] + pv[2];
+    l[1] += pv[1] + pv[3];
+    // P^T B fragments: [0] keys 2cq, 2cq+1 of head g, [1] keys 8 + 2cq, 8 + 2cq + 1
+    const uint32_t pb0 = movmatrix_t(pack_bf16x2(pv[0], pv[1]));
+    const uint32_t pb1 = movmatrix_t(pack_bf16x2(pv[2], pv[3]));
 #pragma unroll
-    for (int nd = 0; nd < 16; nd += 2) {
-      uint32_t v0, v1, v2, v3;
-      ldsm_x4_t(vt + tile_off(vrow, nd + (lane >> 4)), v0, v1, v2, v3);
-      mma16816(o[nd], pa[0], pa[1], pa[2], pa[3], v0, v1);
-      mma16816(o[nd + 1], pa[0], pa[1], pa[2], pa[3], v2, v3);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar(kStages + s));
+    for (int mt = 0; mt < 8; ++mt)
+      mma16816(o[mt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb0, pb1);
   }
   if (!ok) {
     *abort_s = 1;
     atomicOr(p.status, kStatusTimeout);
     return;
   }
-  // row sums across the 4 threads of a row group
+  // column sums across the 8 row groups
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 1);
-    l[rr] += __shfl_xor_sync(0xffffffffu, l[rr], 2);
+  for (int e = 0; e < 2; ++e) {
+    l[e] += __shfl_xor_sync(0xffffffffu, l[e], 4);
+    l[e] += __shfl_xor_sync(0xffffffffu, l[e], 8);
+    l[e] += __shfl_xor_sync(0xffffffffu, l[e], 16);
   }
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int row = g + 8 * rr;
-    if (row >= rows) continue;
-    float *dst = p.ws + ((static_cast<int64_t>(b) * p.Hq + hk * p.group + row) * p.n_chunks + c) *
+  for (int e = 0; e < 2; ++e) {
+    const int h = 2 * cq + e;
+    if (h >= heads) continue;
+    float *dst = p.ws + ((static_cast<int64_t>(b) * p.Hq + hk * p.group + h) * p.n_chunks + c) *
                             kDecodePartialFloats;
 #pragma unroll
-    for (int nd = 0; nd < 16; ++nd) {
-      dst[8 * nd + 2 * cq] = o[nd][2 * rr];
-      dst[8 * nd + 2 * cq + 1] = o[nd][2 * rr + 1];
+    for (int mt = 0; mt < 8; ++mt) {
+      dst[16 * mt + g] = o[mt][e];
+      dst[16 * mt + g + 8] = o[mt][2 + e];
     }
-    if (cq == 0) {
-      dst[kD] = m[rr];
-      dst[kD + 1] = l[rr];
+    if (g == 0) {
+      dst[kD] = m[e];
+      dst[kD + 1] = l[e];
     }
   }
   // the combine kernel (a programmatic dependent) may be scheduled once every
@@ -517,6 +554,7 @@ cudaError_t launch_decode_mma(const DecodeArgs &a, unsigned *status, cudaStream_
   p.n_chunks = a.n_chunks;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.skip_first_arrival = a.debug_skip_arrival ? 1 : 0;
+  p.g_magic = a.G >= 2 ? (~0ull / static_cast<unsigned long long>(a.G)) + 1ull : 0ull;
   dim3 grid(a.n_chunks, a.B);
   bifocal_decode_mma_kernel<<<grid, kThreads, kSmemAlloc, s>>>(mk, mv, p);
   cudaError_t e = cudaGetLastError();

@@ -108,7 +108,7 @@ def _decode(lib, **kw):
     (dict(kc=FAKE + 4), INVALID),
     (dict(w_local=-3), INVALID),
     (dict(flags=2), INVALID),
-    (dict(Hq=34, Hkv=2, flags=1 << 31), UNSUPPORTED),  # group 17: no tensor-core kernel
+    (dict(Hq=18, Hkv=2, flags=1 << 31), UNSUPPORTED),  # group 9: no tensor-core kernel
 ])
 def test_decode_rejects(lib, kw, code):
     assert _decode(lib, **kw) == code
