@@ -40,7 +40,7 @@ METRIC = "bifocal prefill TFLOP/s & % bf16 peak; decode KV-read GB/s & % HBM"
 # DRAM bytes (read + write) of one full-size launch of the prefill kernel,
 # from ncu (dram__bytes_read.sum + dram__bytes_write.sum, one pass) on B200.
 # Must be re-measured (or set to None) whenever that kernel changes.
-PREFILL_TRAFFIC_BYTES = 79.507e9 + 1.067e9
+PREFILL_TRAFFIC_BYTES = None
 PREFILL_CFG = "qwen3_8b_L131072"
 DECODE_CFG = "qwen3_8b_decode_n131072"
 
@@ -334,7 +334,7 @@ def run_cuda(args):
         },
         "roofline": {
             "bound": "tensor",
-            "kernel": "bifocal_prefill_sm100_kernel (+ key-rotation pass, timed together)",
+            "kernel": "bifocal_prefill_sm100_x2_kernel (+ key-rotation pass, timed together)",
             "achieved": round(achieved, 2),
             "peak": bf16_sust,
             "peak_kind": f"bf16 dense, sustained, {src}",

@@ -290,13 +290,13 @@ jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v, voi
   if (e != cudaSuccess) return cuda_fail(e, "key rotation launch");
   a.kstd = need_std ? kstd : nullptr;
   a.krem = need_rem ? krem : nullptr;
-  // The two-head kernel is opt-in while it is slower than the one-tile kernel.
-  static const bool use_x2 = [] {
-    const char *v = std::getenv("JL_PREFILL_X2");
-    return v != nullptr && v[0] == '1';
-  }();
-  e = (use_x2 && prefill_x2_supported(a)) ? launch_prefill_sm100_x2(a, s)
-                                          : launch_prefill_sm100(a, s);
+  // Two query heads of one kv head per CTA where the group size is even (the
+  // faster kernel); JL_PREFILL_KERNEL=one selects the one-tile kernel, read
+  // on every call so that tests can cover both.
+  const char *kv = std::getenv("JL_PREFILL_KERNEL");
+  const bool one_tile = kv != nullptr && std::strcmp(kv, "one") == 0;
+  e = (!one_tile && prefill_x2_supported(a)) ? launch_prefill_sm100_x2(a, s)
+                                             : launch_prefill_sm100(a, s);
   return e == cudaSuccess ? JL_OK : cuda_fail(e, "prefill launch");
 }
 

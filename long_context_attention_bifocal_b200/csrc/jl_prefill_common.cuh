@@ -136,5 +136,25 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + static_cast<int>(static_cast<unsigned>(e) << 23));
 }
 
+// The same 2^x on a pair of fp32 values with packed fp32 arithmetic: clamp,
+// one round-down add for floor, the cubic in three packed FMAs, and the
+// exponent added to the bits of each result.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  const uint64_t kMagic2 = 0x4B4000004B400000ull;  // (1.5 * 2^23, 1.5 * 2^23)
+  float x0, x1;
+  sm100::f2_unpack(x2, x0, x1);
+  x2 = sm100::f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  const uint64_t t2 = sm100::f2_add_rd(x2, kMagic2);  // magic + floor(x), exact
+  const uint64_t f2 = sm100::f2_sub(x2, sm100::f2_sub(t2, kMagic2));
+  // the cubic's coefficients as fp32 bit patterns, one copy per half
+  uint64_t p2 = sm100::f2_fma(0x3DA0145E3DA0145Eull, f2, 0x3E67E0583E67E058ull);
+  p2 = sm100::f2_fma(p2, f2, 0x3F32055E3F32055Eull);
+  p2 = sm100::f2_fma(p2, f2, 0x3F8000003F800000ull);
+  // magic's low bits are zero, so (t << 23) is floor(x) << 23 modulo 2^32
+  const uint32_t t_lo = static_cast<uint32_t>(t2), t_hi = static_cast<uint32_t>(t2 >> 32);
+  const uint32_t p_lo = static_cast<uint32_t>(p2), p_hi = static_cast<uint32_t>(p2 >> 32);
+  return (static_cast<uint64_t>(p_hi + (t_hi << 23)) << 32) | (p_lo + (t_lo << 23));
+}
+
 }  // namespace prefill
 }  // namespace jl

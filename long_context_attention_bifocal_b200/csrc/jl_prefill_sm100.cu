@@ -41,6 +41,7 @@
 
 #include <climits>
 #include <mutex>
+#include <type_traits>
 
 #include "jl_prefill_common.cuh"
 
@@ -51,14 +52,13 @@ using namespace sm100;
 using namespace prefill;
 
 // shared-memory layout (bytes from the 1 KiB-aligned base), barriers, TMEM
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kThreads = 192;
 
 constexpr uint32_t kOffQ = 0;  // the Q variant of the current phase
 constexpr uint32_t kOffK = kOffQ + kTileBytes;
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
-constexpr uint32_t kOffP = kOffV + kStages * kTileBytes;  // [2] P buffers
-constexpr uint32_t kOffBar = kOffP + 2 * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
 
 enum : int {
   kBarQFull = 0,  // phase 0: first Q variant; phase 1: Q_std after the remote passes
@@ -83,12 +83,15 @@ static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmS0 = 0, kTmS1 = 128, kTmO = 256;
+constexpr uint32_t kTmP = 384;  // [2] P buffers, 64 columns each (bf16 pairs)
 
-// pairs (of each 4 in an 8-key chunk) whose 2^x runs on the FMA pipe
-#ifndef JL_POLY_PAIRS
-#define JL_POLY_PAIRS 0
+// one column pair in kPolyEvery takes 2^x on the FMA pipe (unmasked tiles);
+// a value above 16 keeps every exponential on the MUFU unit.  Off by default:
+// on a B200 at L = 131072 one pair in 8 costs 2% and one in 2 costs 9%.
+#ifndef JL_POLY_EVERY
+#define JL_POLY_EVERY 1000
 #endif
-constexpr int kPolyPairs = JL_POLY_PAIRS;
+constexpr int kPolyEvery = JL_POLY_EVERY;
 
 struct KParams {
   const __nv_bfloat16 *q;
@@ -239,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 128; ++e) mx[e & 7] = fmaxf(mx[e & 7], s[e]);
+        for (int e = 0; e < 128; e += 2) mx[(e >> 1) & 7] = fmax3(mx[(e >> 1) & 7], s[e], s[e + 1]);
         const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
                          p.scale_log2;  // scale > 0 keeps the order
@@ -273,40 +276,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(lane_base + kTmO + 32 * c, o);
           }
         }
-        // P = 2^(s * scale * log2(e) - m), one FFMA per element (-inf gives 0),
-        // stored as bf16 8 keys at a time into P buffer it & 1; that buffer was
-        // last read by the product of pass it-2, complete before this S.
+        // P = 2^(s * scale * log2(e) - m) on pairs of columns with packed fp32
+        // arithmetic (-inf gives 0); in unmasked tiles one pair in kPolyEvery
+        // takes the FMA-pipe polynomial instead of two MUFU exponentials, so
+        // the MUFU unit is not the only bound.  Column j of the P buffer (TMEM,
+        // bf16) holds keys (2j, 2j+1); that buffer was last read by the
+        // product of pass it-2, complete before this S.
         const bool plain = !causal && mk == kMaskNone;
         const float neg_mu = (m == -INFINITY) ? 0.f : -m;
-        float rsum[8];
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2_pack(neg_mu, neg_mu);
+        uint64_t rsum2[4] = {0ull, 0ull, 0ull, 0ull};
+        const uint32_t pcol = lane_base + kTmP + 64 * pbuf;
+        // two copies of the loop so that neither has a branch inside
+        auto exp_row = [&](auto with_poly) {
 #pragma unroll
-        for (int a = 0; a < 8; ++a) rsum[a] = 0.f;
-        uint8_t *pdst = smem + kOffP + pbuf * kTileBytes;
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = fmaf(s[8 * c + 2 * e], p.scale_log2, neg_mu);
-            const float x1 = fmaf(s[8 * c + 2 * e + 1], p.scale_log2, neg_mu);
-            float p0, p1;
-            if (plain && e < kPolyPairs) {
-              p0 = exp2_poly(x0);
-              p1 = exp2_poly(x1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
+            for (int q = 0; q < 16; ++q) {
+              const int j = 16 * c4 + q;
+              const uint64_t x2 = f2_fma(f2_pack(s[2 * j], s[2 * j + 1]), sc2, nm2);
+              uint64_t p2;
+              if (decltype(with_poly)::value && (q % kPolyEvery) == kPolyEvery - 1) {
+                p2 = exp2_poly2(x2);
+              } else {
+                float a, b;
+                f2_unpack(x2, a, b);
+                p2 = f2_pack(ex2_approx(a), ex2_approx(b));
+              }
+              rsum2[q & 3] = f2_add(rsum2[q & 3], p2);
+              float p0, p1;
+              f2_unpack(p2, p0, p1);
+              pk[q] = pack_bf16x2(p0, p1);
             }
-            rsum[(2 * c + e) & 7] += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
+            tmem_st16_nowait(pcol + 16 * c4, pk);
           }
-          *reinterpret_cast<uint4 *>(pdst + (c >> 3) * kHalfBytes + swz(r, c & 7)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        };
+        if (plain)
+          exp_row(std::true_type{});
+        else
+          exp_row(std::false_type{});
+        tmem_wait_st();
+        float rs;
+        {
+          const uint64_t r2 = f2_add(f2_add(rsum2[0], rsum2[1]), f2_add(rsum2[2], rsum2[3]));
+          float r0, r1;
+          f2_unpack(r2, r0, r1);
+          rs = r0 + r1;
         }
-        const float rs = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) +
-                         ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
         l = l * alpha + rs;
-        fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar(kBarPFull + pbuf));
         ++it;
@@ -397,15 +416,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             return false;
           if (!mbar_wait(bar(kBarVFull + s), ph, abort_s, abort_g, kTimeoutNs)) return false;
           tc_fence_after();
-          const uint32_t pa = sb + kOffP + pbuf * kTileBytes;
+          const uint32_t pa = tmem + kTmP + 64 * pbuf;  // P from TMEM, 8 columns per step
           const uint32_t vb = sb + kOffV + s * kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {  // 16 keys per step
-            const uint32_t a_off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
             const uint32_t b_off = kk * 2048;  // 16 key rows of 128 B
-            umma_bf16(tmem + kTmO, sdesc_sw128(pa + a_off, 16, 1024),
-                      sdesc_sw128(vb + b_off, kHalfBytes, 1024), idesc_pv,
-                      (tt > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16_ts(tmem + kTmO, pa + 8 * kk, sdesc_sw128(vb + b_off, kHalfBytes, 1024),
+                         idesc_pv, (tt > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(bar(kBarODone + pbuf));
           umma_commit(bar(kBarVEmpty + s));

@@ -38,6 +38,7 @@
 
 #include <climits>
 #include <mutex>
+#include <type_traits>
 
 #include "jl_prefill_common.cuh"
 
@@ -79,11 +80,17 @@ constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
+
+// one column pair in kPolyEvery takes 2^x on the FMA pipe (unmasked tiles);
+// a value above 16 keeps every exponential on the MUFU unit.  Off by default:
+// measured on a B200 at L = 131072, every 4th pair costs 2% and every 2nd 12%.
+#ifndef JL_X2_POLY_EVERY
+#define JL_X2_POLY_EVERY 1000
+#endif
+constexpr int kPolyEvery = JL_X2_POLY_EVERY;
 __host__ __device__ constexpr uint32_t tm_s(int t) { return 128u * t; }
 __host__ __device__ constexpr uint32_t tm_o(int t) { return 256u + 128u * t; }
 
-// elements of each 32-column chunk whose 2^x runs on the FMA pipe
-constexpr int kPolyPer32 = 10;
 
 struct KParams {
   const __nv_bfloat16 *q;
@@ -232,24 +239,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (mk == kMaskLocalOnly) v = v && dd < p.w;
           return v;
         };
-        // pass 1 over S: row max of the raw scores, 8 independent chains
+        // pass 1 over S, 64 columns at a time: row max of the raw scores
         float mt;
         {
-          float sv[128];
-          tmem_ld128(s_col, sv);
           float mx[8];
 #pragma unroll
           for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
-          if (plain) {
 #pragma unroll
-            for (int e = 0; e < 128; ++e) mx[e & 7] = fmaxf(mx[e & 7], sv[e]);
-          } else {
+          for (int h = 0; h < 2; ++h) {
+            float sv[64];
+            tmem_ld64(s_col + 64 * h, sv);
+            if (!plain) {
 #pragma unroll
-            for (int e = 0; e < 128; ++e)
-              mx[e & 7] = fmaxf(mx[e & 7], valid(e) ? sv[e] : -INFINITY);
+              for (int e = 0; e < 64; ++e) sv[e] = valid(64 * h + e) ? sv[e] : -INFINITY;
+            }
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) mx[(e >> 1) & 7] = fmax3(mx[(e >> 1) & 7], sv[e], sv[e + 1]);
           }
-          mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+          mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
                p.scale_log2;  // scale > 0 keeps the order
         }
         const float m_new = fmaxf(m, mt);
@@ -279,32 +286,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         float rsum[8];
 #pragma unroll
         for (int a = 0; a < 8; ++a) rsum[a] = 0.f;
+        // one column pair in kPolyEvery of an unmasked tile takes 2^x on the
+        // FMA pipe: the two softmax warpgroups share each SM sub-partition's
+        // MUFU unit, which would otherwise bound this pass.  Two copies of the
+        // loop, so that neither has a branch inside.
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2_pack(neg_mu, neg_mu);
+        auto exp_pass = [&](auto with_poly) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float sv[32];
-          tmem_ld32(s_col + 32 * c, sv);
-          if (!plain) {
+          for (int c = 0; c < 4; ++c) {
+            float sv[32];
+            tmem_ld32(s_col + 32 * c, sv);
+            if (!decltype(with_poly)::value) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) sv[e] = valid(32 * c + e) ? sv[e] : -INFINITY;
-          }
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x0 = fmaf(sv[2 * e], p.scale_log2, neg_mu);
-            const float x1 = fmaf(sv[2 * e + 1], p.scale_log2, neg_mu);
-            float p0, p1;
-            if (plain && 2 * e < kPolyPer32) {
-              p0 = exp2_poly(x0);
-              p1 = exp2_poly(x1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
+              for (int e = 0; e < 32; ++e) sv[e] = valid(32 * c + e) ? sv[e] : -INFINITY;
             }
-            rsum[e & 7] += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              float p0, p1;
+              if (decltype(with_poly)::value && (e % kPolyEvery) == kPolyEvery - 1) {
+                const uint64_t x2 = f2_fma(f2_pack(sv[2 * e], sv[2 * e + 1]), sc2, nm2);
+                f2_unpack(exp2_poly2(x2), p0, p1);
+              } else {
+                p0 = ex2_approx(fmaf(sv[2 * e], p.scale_log2, neg_mu));
+                p1 = ex2_approx(fmaf(sv[2 * e + 1], p.scale_log2, neg_mu));
+              }
+              rsum[e & 7] += p0 + p1;
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+            // chunk c of P lands on S columns [16c, 16c+16), read by chunks <= c/2
+            tmem_st16_nowait(s_col + 16 * c, pk);
           }
-          tmem_st16(s_col + 16 * c, pk);
-        }
+        };
+        if (plain)
+          exp_pass(std::true_type{});
+        else
+          exp_pass(std::false_type{});
+        tmem_wait_st();
         const float rs = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) +
                          ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
         l = l * alpha + rs;
@@ -389,64 +408,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto wait = [&](int i, uint32_t parity) {
           return mbar_wait(bar(i), parity, abort_s, abort_g, kTimeoutNs);
         };
+        // Issue order (one thread, so the tensor core runs it in order):
+        //   S_0(0) S_1(0) | PV_0(0) S_0(1) PV_1(0) S_1(1) | PV_0(1) S_0(2) ...
+        // S_t(j+1) overwrites the columns P_t(j) lives in; it is issued after
+        // PV_t(j), which has read them.  While head t's softmax runs on S_t(j),
+        // the tensor core works on head 1-t.
         PassIter it;
         it.begin(qt, p.w);
         bool ok = true;
-        int j = 0, qphase = 0;
-        int prev_kind = it.kind();
-        while (ok && !it.done()) {
-          const int kind = it.kind();
-          const int s = j % kStages;
-          const uint32_t ph = (j / kStages) & 1;
-          if (j == 0 || kind != prev_kind) {
-            // the Q variant this pass needs is in shared memory
-            ok = wait(kBarQReady + 0, qphase & 1) && wait(kBarQReady + 1, qphase & 1);
-            ++qphase;
+        int qphase[2] = {0, 0};
+        auto issue_s = [&](int t, int jj, int kind_changed) -> bool {
+          const int s = jj % kStages;
+          if (kind_changed) {
+            if (!wait(kBarQReady + t, qphase[t] & 1)) return false;
+            ++qphase[t];
           }
-          ok = ok && wait(kBarKFull + s, ph);
-          if (!ok) break;
+          if (t == 0 && !wait(kBarKFull + s, (jj / kStages) & 1)) return false;
+          tc_fence_after();
+          const uint32_t a0 = sb + (t == 0 ? kOffQ0 : kOffQ1);
           const uint32_t b0 = sb + kOffK + s * kTileBytes;
-          for (int t = 0; t < 2; ++t) {
-            // S_t holds P_t of the previous pass until that product completed
-            if (j > 0 && !wait(kBarODone + t, (j - 1) & 1)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t a0 = sb + (t == 0 ? kOffQ0 : kOffQ1);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-              umma_bf16(tmem + tm_s(t), sdesc_sw128(a0 + off, 16, 1024),
-                        sdesc_sw128(b0 + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-            }
-            umma_commit(bar(kBarSFull + t));
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+            umma_bf16(tmem + tm_s(t), sdesc_sw128(a0 + off, 16, 1024),
+                      sdesc_sw128(b0 + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
           }
-          if (!ok) break;
-          umma_commit(bar(kBarKEmpty + s));
-          if (!wait(kBarVFull + s, ph)) {
-            ok = false;
-            break;
-          }
+          umma_commit(bar(kBarSFull + t));
+          if (t == 1) umma_commit(bar(kBarKEmpty + s));  // both heads' S issued
+          return true;
+        };
+        auto issue_pv = [&](int t, int jj) -> bool {
+          const int s = jj % kStages;
+          if (!wait(kBarPFull + t, jj & 1)) return false;
+          if (t == 0 && !wait(kBarVFull + s, (jj / kStages) & 1)) return false;
+          tc_fence_after();
           const uint32_t vb = sb + kOffV + s * kTileBytes;
-          for (int t = 0; t < 2; ++t) {
-            if (!wait(kBarPFull + t, j & 1)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {  // 16 keys per step, P_t from TMEM
-              umma_bf16_ts(tmem + tm_o(t), tmem + tm_s(t) + 8 * kk,
-                           sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idesc_pv,
-                           (j > 0 || kk > 0) ? 1u : 0u);
-            }
-            umma_commit(bar(kBarODone + t));
-          }
-          if (!ok) break;
-          umma_commit(bar(kBarVEmpty + s));
-          prev_kind = kind;
+          for (int kk = 0; kk < 8; ++kk)  // 16 keys per step, P_t from TMEM
+            umma_bf16_ts(tmem + tm_o(t), tmem + tm_s(t) + 8 * kk,
+                         sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idesc_pv,
+                         (jj > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar(kBarODone + t));
+          if (t == 1) umma_commit(bar(kBarVEmpty + s));
+          return true;
+        };
+        int j = 0;
+        int kind = it.kind();
+        ok = issue_s(0, 0, 1) && issue_s(1, 0, 1);
+        while (ok && !it.done()) {
           it.next();
+          const bool more = !it.done();
+          const int next_kind = more ? it.kind() : kind;
+          const int changed = more && next_kind != kind;
+          ok = issue_pv(0, j) && (!more || issue_s(0, j + 1, changed)) && issue_pv(1, j) &&
+               (!more || issue_s(1, j + 1, changed));
+          kind = next_kind;
           ++j;
         }
         if (!ok) raise_abort(abort_s, p.status);

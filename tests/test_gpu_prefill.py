@@ -75,6 +75,14 @@ def test_bf16_small_all_rows(jl, oracle_mod, case):
                  max_abs=parity.BF16_MAX_ABS, mean_abs=parity.BF16_MEAN_ABS, what=str(case))
 
 
+@pytest.mark.parametrize("case", SMALL, ids=[f"B{c[0]}L{c[1]}H{c[2]}x{c[3]}wp{c[4]}wl{c[5]}s{c[6]}" for c in SMALL])
+def test_bf16_small_all_rows_one_tile_kernel(jl, oracle_mod, case, monkeypatch):
+    """The same cases on the one-query-tile kernel (the default takes two query
+    heads per CTA whenever the group size is even)."""
+    monkeypatch.setenv("JL_PREFILL_KERNEL", "one")
+    test_bf16_small_all_rows(jl, oracle_mod, case)
+
+
 def test_bf16_g1_bitwise_plain(jl):
     """G = 1 takes exactly the non-bifocal path."""
     q, k, v = W.prefill_inputs(1, 777, 4, 2, 128, seed=7)
@@ -110,6 +118,15 @@ FULL = ["qwen3_1p7b_L65536", "qwen3_8b_L131072", "qwen3_4b_L16384", "qwen3_4b_L3
 
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_sampled_rows(jl, oracle_mod, name):
+    full_size_sampled_rows(jl, oracle_mod, name)
+
+
+def test_full_size_sampled_rows_one_tile_kernel(jl, oracle_mod, monkeypatch):
+    monkeypatch.setenv("JL_PREFILL_KERNEL", "one")
+    full_size_sampled_rows(jl, oracle_mod, "qwen3_8b_L131072")
+
+
+def full_size_sampled_rows(jl, oracle_mod, name):
     cfg = W.PREFILL[name]
     B, L, Hq, Hkv, D = cfg["B"], cfg["L"], cfg["Hq"], cfg["Hkv"], cfg["D"]
     q, k, v = W.prefill_inputs(B, L, Hq, Hkv, D, value_scale=cfg["value_scale"],
