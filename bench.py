@@ -259,6 +259,15 @@ def run_cuda(args):
     dec_bif, dec_plain = interleaved_ms(lambda: decode(0), lambda: decode(jl.NO_BIFOCAL), 100)
     pre_plain = avg_ms(lambda: prefill(jl.NO_BIFOCAL), max(1, min(3, args.steps)))
     pre_bif = avg_ms(lambda: prefill(0), max(1, min(3, args.steps)))
+    # the pages' unfused three-call formulation of the same prefill (A + B - C)
+    ws3 = torch.empty(jl.prefill_3pass_workspace_size(B, L, Hq, Hkv, D), dtype=torch.uint8,
+                      device=dev)
+    out3 = torch.empty_like(out)
+    lse3 = torch.empty_like(lse)
+    pre_3pass = avg_ms(lambda: jl.bifocal_prefill_3pass(q, k, v, out=out3, lse=lse3,
+                                                        workspace=ws3, **kwp),
+                       max(1, min(3, args.steps)))
+    del ws3, out3, lse3
     jl.check_device_status()
 
     # ---------------- end to end through the public API, host buffers ----------
@@ -325,6 +334,11 @@ def run_cuda(args):
             "us_per_call_in_step": round(dec_sum / args.steps * 1e3, 2),
             "frac_hbm": round(dec_gbs / world / hbm, 4),
             "overhead_vs_no_bifocal": round(dec_bif / dec_plain - 1.0, 4),
+        },
+        "prefill_unfused_3pass": {
+            "ms_per_call": round(pre_3pass, 3),
+            "tflops_effective": round(flops / (pre_3pass / 1e3) / 1e12, 2),
+            "fused_speedup": round(pre_3pass / pre_bif, 4),
         },
         "prefill": {
             "ms_per_call": round(pre_launch_ms, 3),

@@ -119,6 +119,32 @@ jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v,
                                 void *workspace, size_t workspace_bytes,
                                 jl_stream_t stream);
 
+/*
+ * The same bifocal prefill through the pages' unfused formulation, kept to
+ * measure the fused kernel against it and as a second GPU check of the
+ * inclusion-exclusion identity (bittide paper summary §3.2; techwalker
+ * explainer §四): three attention calls and a LogSumExp merge,
+ *   A = causal attention with every pair at remapped positions (f(q), f(k)),
+ *   B = the local window (0 <= q - k < w_local) at original positions,
+ *   C = the same window at remapped positions,
+ *   out = (e^lse_A O_A + e^lse_B O_B - e^lse_C O_C) / (e^lse_A + e^lse_B - e^lse_C),
+ *   lse = ln(e^lse_A + e^lse_B - e^lse_C).
+ * Arguments, layouts and results are those of jl_bifocal_prefill (bf16,
+ * D == 128; flags: JL_FLAG_NO_BIFOCAL).  A is written to out / lse and merged
+ * in place; O_B, O_C (bf16) and their lse live in the workspace, so the merge
+ * sees outputs rounded to bf16 (the fused kernel has no such step).
+ * workspace: device memory of at least
+ * jl_bifocal_prefill_3pass_workspace_size() bytes, 256-byte aligned
+ * (required).  With w_local = 0 the window is empty and out = A.
+ */
+size_t jl_bifocal_prefill_3pass_workspace_size(int B, int L, int Hq, int Hkv, int D);
+jl_status jl_bifocal_prefill_3pass(const void *q, const void *k, const void *v,
+                                   void *out, float *lse, int B, int L, int Hq,
+                                   int Hkv, int D, int w_local, int w_pretrained,
+                                   double rope_base, unsigned flags,
+                                   void *workspace, size_t workspace_bytes,
+                                   jl_stream_t stream);
+
 /* Bytes of workspace jl_bifocal_decode needs for these sizes. */
 size_t jl_bifocal_decode_workspace_size(int B, int Hq, int Hkv, int D, int pos);
 

@@ -16,6 +16,7 @@ import torch
 __all__ = [
     "NO_BIFOCAL", "DEBUG_SKIP_ARRIVE", "JetLongError", "group_size", "bifocal_prefill",
     "prefill_workspace_size", "decode_workspace_size", "bifocal_decode",
+    "bifocal_prefill_3pass", "prefill_3pass_workspace_size",
     "bifocal_decode_noalloc",
     "check_device_status", "finalize", "library_path", "load",
 ]
@@ -63,6 +64,10 @@ def load():
     L.jl_bifocal_prefill_ex.restype = i
     L.jl_bifocal_prefill_ex.argtypes = [p, p, p, p, p, i, i, i, i, i, i, i, d, i,
                                         ctypes.c_float, u, p, sz, p]
+    L.jl_bifocal_prefill_3pass_workspace_size.restype = sz
+    L.jl_bifocal_prefill_3pass_workspace_size.argtypes = [i, i, i, i, i]
+    L.jl_bifocal_prefill_3pass.restype = i
+    L.jl_bifocal_prefill_3pass.argtypes = [p, p, p, p, p, i, i, i, i, i, i, i, d, u, p, sz, p]
     L.jl_bifocal_decode_workspace_size.restype = sz
     L.jl_bifocal_decode_workspace_size.argtypes = [i, i, i, i, i]
     L.jl_bifocal_decode.restype = i
@@ -148,6 +153,37 @@ def bifocal_prefill(q, k, v, *, w_local, w_pretrained, rope_base, out=None, lse=
             int(w_local), int(w_pretrained), float(rope_base),
             _BF16 if dtype == torch.bfloat16 else _F32, float(softmax_scale),
             int(flags), ws_ptr, ws_bytes, _stream(stream)))
+    return out, lse
+
+
+def prefill_3pass_workspace_size(B, L, Hq, Hkv, D) -> int:
+    return int(load().jl_bifocal_prefill_3pass_workspace_size(B, L, Hq, Hkv, D))
+
+
+def bifocal_prefill_3pass(q, k, v, *, w_local, w_pretrained, rope_base, out=None, lse=None,
+                          flags=0, workspace=None, stream=None):
+    """The pages' unfused three-call formulation (A + B - C, LSE merge) of the
+    same bifocal prefill; bf16, D=128.  Returns (out, lse) like bifocal_prefill."""
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _need(q, "q", torch.bfloat16)
+    _need(k, "k", torch.bfloat16, (B, L, Hkv, D))
+    _need(v, "v", torch.bfloat16, (B, L, Hkv, D))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.bfloat16, (B, L, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq, L))
+    if workspace is None:
+        workspace = torch.empty(prefill_3pass_workspace_size(B, L, Hq, Hkv, D),
+                                dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", torch.uint8)
+    with torch.cuda.device(q.device):
+        _check(load().jl_bifocal_prefill_3pass(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, L, Hq, Hkv, D, int(w_local),
+            int(w_pretrained), float(rope_base), int(flags), _ptr(workspace),
+            workspace.numel(), _stream(stream)))
     return out, lse
 
 

@@ -195,6 +195,16 @@ jl_status check_common(int B, int L, int Hq, int Hkv, int D, int w_local, int w_
   return JL_OK;
 }
 
+// Two query heads of one kv head per CTA where the group size is even (the
+// faster kernel); JL_PREFILL_KERNEL=one selects the one-tile kernel, read on
+// every call so that tests can cover both.
+cudaError_t launch_attention(const jl::PrefillArgs &a, cudaStream_t s) {
+  const char *kv = std::getenv("JL_PREFILL_KERNEL");
+  const bool one_tile = kv != nullptr && std::strcmp(kv, "one") == 0;
+  return (!one_tile && jl::prefill_x2_supported(a)) ? jl::launch_prefill_sm100_x2(a, s)
+                                                    : jl::launch_prefill_sm100(a, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -290,13 +300,7 @@ jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v, voi
   if (e != cudaSuccess) return cuda_fail(e, "key rotation launch");
   a.kstd = need_std ? kstd : nullptr;
   a.krem = need_rem ? krem : nullptr;
-  // Two query heads of one kv head per CTA where the group size is even (the
-  // faster kernel); JL_PREFILL_KERNEL=one selects the one-tile kernel, read
-  // on every call so that tests can cover both.
-  const char *kv = std::getenv("JL_PREFILL_KERNEL");
-  const bool one_tile = kv != nullptr && std::strcmp(kv, "one") == 0;
-  e = (!one_tile && prefill_x2_supported(a)) ? launch_prefill_sm100_x2(a, s)
-                                             : launch_prefill_sm100(a, s);
+  e = launch_attention(a, s);
   return e == cudaSuccess ? JL_OK : cuda_fail(e, "prefill launch");
 }
 
@@ -305,6 +309,101 @@ jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v, void *
                              int w_pretrained, double rope_base, jl_stream_t stream) {
   return jl_bifocal_prefill_ex(q, k, v, out, lse, B, L, Hq, Hkv, D, w_local, w_pretrained,
                                rope_base, JL_BF16, 0.f, 0u, nullptr, 0, stream);
+}
+
+size_t jl_bifocal_prefill_3pass_workspace_size(int B, int L, int Hq, int Hkv, int D) {
+  if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || D < 2) return 0;
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t o = up(static_cast<size_t>(B) * L * Hq * D * sizeof(__nv_bfloat16));
+  const size_t l = up(static_cast<size_t>(B) * Hq * L * sizeof(float));
+  return prefill_ws_bytes(B, L, Hkv, D) + 2 * o + 2 * l;
+}
+
+jl_status jl_bifocal_prefill_3pass(const void *q, const void *k, const void *v, void *out,
+                                   float *lse, int B, int L, int Hq, int Hkv, int D,
+                                   int w_local, int w_pretrained, double rope_base,
+                                   unsigned flags, void *workspace, size_t workspace_bytes,
+                                   jl_stream_t stream) {
+  g_last_error.clear();
+  jl_status st = check_common(B, L, Hq, Hkv, D, w_local, w_pretrained, rope_base);
+  if (st != JL_OK) return st;
+  if (!q || !k || !v || !out || !lse || !workspace)
+    return fail(JL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(JL_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(JL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL)) != 0)
+    return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if (D != 128) return fail(JL_ERR_UNSUPPORTED, "the three-call path supports head dim 128 (got %d)", D);
+  if (static_cast<long long>((L + 127) / 128) * B * Hq >= (1LL << 31))
+    return fail(JL_ERR_UNSUPPORTED, "problem too large for one launch");
+  const size_t need = jl_bifocal_prefill_3pass_workspace_size(B, L, Hq, Hkv, D);
+  if (workspace_bytes < need)
+    return fail(JL_ERR_INVALID_ARG, "workspace too small: %zu bytes, need %zu", workspace_bytes,
+                need);
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long G = (flags & JL_FLAG_NO_BIFOCAL) ? 1 : group_size_ll(L, w_pretrained);
+  PrefillArgs a;
+  a.q = q;
+  a.v = v;
+  a.B = B;
+  a.L = L;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.D = D;
+  a.G = static_cast<int>(G);
+  a.scale = static_cast<float>(1.0 / std::sqrt(D));
+  st = rope_table(D, rope_base, L, s, &a.table);
+  if (st != JL_OK) return st;
+  st = status_word(&a.status);
+  if (st != JL_OK) return st;
+
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  char *ws = static_cast<char *>(workspace);
+  const size_t kb = prefill_ws_bytes(B, L, Hkv, D);
+  __nv_bfloat16 *kstd = reinterpret_cast<__nv_bfloat16 *>(ws);
+  __nv_bfloat16 *krem = reinterpret_cast<__nv_bfloat16 *>(ws + kb / 2);
+  const size_t ob = up(static_cast<size_t>(B) * L * Hq * D * sizeof(__nv_bfloat16));
+  const size_t lb = up(static_cast<size_t>(B) * Hq * L * sizeof(float));
+  __nv_bfloat16 *o_b = reinterpret_cast<__nv_bfloat16 *>(ws + kb);
+  __nv_bfloat16 *o_c = reinterpret_cast<__nv_bfloat16 *>(ws + kb + ob);
+  float *l_b = reinterpret_cast<float *>(ws + kb + 2 * ob);
+  float *l_c = reinterpret_cast<float *>(ws + kb + 2 * ob + lb);
+
+  cudaError_t e = launch_rotate_keys(static_cast<const __nv_bfloat16 *>(k),
+                                     w_local > 0 ? kstd : nullptr, krem, a.table, B, L, Hkv, D,
+                                     a.G, s);
+  if (e != cudaSuccess) return cuda_fail(e, "key rotation launch");
+  // A: every pair at remapped positions, into out / lse
+  a.out = out;
+  a.lse = lse;
+  a.kstd = nullptr;
+  a.krem = krem;
+  a.w_eff = 0;
+  a.band = 0;
+  e = launch_attention(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch (A)");
+  if (w_local == 0) return JL_OK;  // empty window: B and C have no pairs
+  // B: the local window at original positions; C: the same window remapped
+  a.w_eff = w_local;
+  a.kstd = kstd;
+  a.krem = nullptr;
+  a.band = 1;
+  a.out = o_b;
+  a.lse = l_b;
+  e = launch_attention(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch (B)");
+  a.kstd = nullptr;
+  a.krem = krem;
+  a.band = 2;
+  a.out = o_c;
+  a.lse = l_c;
+  e = launch_attention(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch (C)");
+  e = launch_lse_merge(static_cast<__nv_bfloat16 *>(out), lse, o_b, l_b, o_c, l_c, B, L, Hq, s);
+  return e == cudaSuccess ? JL_OK : cuda_fail(e, "merge launch");
 }
 
 size_t jl_bifocal_decode_workspace_size(int B, int Hq, int Hkv, int D, int pos) {

@@ -59,6 +59,7 @@ struct PrefillArgs {
   float scale;        // softmax scale
   RopeTable table;
   unsigned *status;
+  int band = 0;       // 0: bifocal rule; 1 / 2: only the local window, standard / remapped
 };
 
 cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s);
@@ -95,6 +96,11 @@ void decode_plan(int B, int Hq, int Hkv, int pos, int far_end, int *chunk,
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 // merges a.n_chunks split partials of a.ws into a.out and a.lse
 cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t s);
+
+// In place: out/lse hold call A; returns the LSE merge of A + B - C.
+cudaError_t launch_lse_merge(__nv_bfloat16 *out, float *lse, const __nv_bfloat16 *ob,
+                             const float *lb, const __nv_bfloat16 *oc, const float *lc, int B,
+                             int L, int Hq, cudaStream_t s);
 
 // TMA-staged tensor-core decode (all kv heads of a key chunk per CTA):
 // needs D == 128, Hkv <= 8 and Hq / Hkv <= 16.

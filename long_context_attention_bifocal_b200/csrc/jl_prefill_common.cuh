@@ -23,6 +23,10 @@ constexpr uint32_t kHalfBytes = kTileBytes / 2;  // 64 columns (128 B rows)
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 
 enum : int { kStd = 0, kRem = 1 };
+// Pass selection: the bifocal rule (every pair in its class), or only the
+// local window with one RoPE class for every pair in it (the B and C calls of
+// the unfused three-call formulation).
+enum : int { kBandNone = 0, kBandStd = 1, kBandRem = 2 };
 enum : int { kMaskNone = 0, kMaskFarOnly = 1, kMaskLocalOnly = 2 };
 
 // The pass schedule of query tile i.  Kv tile j <= i is at tile distance
@@ -42,8 +46,10 @@ struct PassIter {
   int a, b;      // last tile with a remote pair (-1: none), first with a local pair
   int phase;     // kRem, then kStd
   int j;         // current kv tile
+  int band;      // kBandNone, or only the local passes with one class
 
-  __device__ void begin(int qi, int wl) {
+  __device__ void begin(int qi, int wl, int band_mode = kBandNone) {
+    band = band_mode;
     i = qi;
     w = wl;
     // smallest d with 128d + 127 >= w
@@ -56,7 +62,7 @@ struct PassIter {
       const long long dmax = (static_cast<long long>(wl) + 126) / kBN;
       b = dmax >= qi ? 0 : qi - static_cast<int>(dmax);
     }
-    if (a >= 0) {
+    if (a >= 0 && band == kBandNone) {
       phase = kRem;
       j = 0;
     } else {
@@ -65,7 +71,9 @@ struct PassIter {
     }
   }
   __device__ bool done() const { return phase == kStd && j > i; }
-  __device__ int kind() const { return phase; }
+  __device__ int kind() const {
+    return band == kBandNone ? phase : (band == kBandStd ? kStd : kRem);
+  }
   __device__ int mask() const {
     if (phase == kRem) return j >= b ? kMaskFarOnly : kMaskNone;
     return j <= a ? kMaskLocalOnly : kMaskNone;

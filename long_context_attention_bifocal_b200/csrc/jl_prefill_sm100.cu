@@ -100,6 +100,7 @@ struct KParams {
   const float2 *cs;
   unsigned *status;
   int B, L, Hq, Hkv, G, w, n_qtiles;
+  int band;  // kBandNone, kBandStd or kBandRem
   float scale_log2;  // softmax scale * log2(e)
 };
 
@@ -198,13 +199,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       {
         PassIter t0;
-        t0.begin(qt, p.w);
+        t0.begin(qt, p.w, p.band);
         rotate_q(t0.kind() == kRem ? pos_rem : pos_std);
       }
 
       float m = -INFINITY, l = 0.f;
       PassIter t;
-      t.begin(qt, p.w);
+      t.begin(qt, p.w, p.band);
       int it = 0;
       bool ok = true;
       while (!t.done()) {
@@ -369,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_krem);
         prefetch_tmap(&tm_v);
         PassIter t;
-        t.begin(qt, p.w);
+        t.begin(qt, p.w, p.band);
         int kiss = 0, viss = 0;  // loads issued
         while (!t.done()) {
           const int s = kiss % kStages;
@@ -429,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         PassIter t;
-        t.begin(qt, p.w);
+        t.begin(qt, p.w, p.band);
         int it = 0, qphase = 0, prev_kind = t.kind();
         while (ok && !t.done()) {
           const int kind = t.kind();
@@ -544,6 +545,7 @@ cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s) {
   p.Hkv = a.Hkv;
   p.G = a.G;
   p.w = a.w_eff;
+  p.band = a.band;
   p.n_qtiles = (a.L + kBM - 1) / kBM;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * a.Hq;

@@ -99,6 +99,7 @@ struct KParams {
   const float2 *cs;
   unsigned *status;
   int B, L, Hq, Hkv, G, w, n_qtiles;
+  int band;  // kBandNone, kBandStd or kBandRem
   float scale_log2;
 };
 
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int pos_rem = row_ok ? qpos / p.G : 0;
 
       PassIter it;
-      it.begin(qt, p.w);
+      it.begin(qt, p.w, p.band);
       // first Q variant = the class of the first pass
       rotate_q_row(qdst, r, qrow, row_ok, p.cs, it.kind() == kRem ? pos_rem : pos_std);
       fence_proxy_async_smem();
@@ -367,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_krem);
         prefetch_tmap(&tm_v);
         PassIter it;
-        it.begin(qt, p.w);
+        it.begin(qt, p.w, p.band);
         int kiss = 0, viss = 0;
         while (!it.done()) {
           const int s = kiss % kStages;
@@ -414,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // PV_t(j), which has read them.  While head t's softmax runs on S_t(j),
         // the tensor core works on head 1-t.
         PassIter it;
-        it.begin(qt, p.w);
+        it.begin(qt, p.w, p.band);
         bool ok = true;
         int qphase[2] = {0, 0};
         auto issue_s = [&](int t, int jj, int kind_changed) -> bool {
@@ -539,6 +540,7 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
   p.Hkv = a.Hkv;
   p.G = a.G;
   p.w = a.w_eff;
+  p.band = a.band;
   p.n_qtiles = (a.L + kBM - 1) / kBM;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * (a.Hq / 2);

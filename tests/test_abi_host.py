@@ -130,3 +130,35 @@ def test_product_path_has_no_oracle_or_fallback():
         if name.endswith(".py"):
             src = open(os.path.join(pkg, name)).read()
             assert "import oracle" not in src and "from oracle" not in src, name
+
+
+def _prefill_3pass(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, B=1, L=256, Hq=4, Hkv=2, D=128,
+             w_local=64, w_pretrained=128, base=1e6, flags=0, ws=FAKE, ws_bytes=1 << 32)
+    a.update(kw)
+    return lib.jl_bifocal_prefill_3pass(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"],
+                                        a["L"], a["Hq"], a["Hkv"], a["D"], a["w_local"],
+                                        a["w_pretrained"], a["base"], a["flags"], a["ws"],
+                                        a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=64), UNSUPPORTED),
+    (dict(ws=None), INVALID),
+    (dict(ws=FAKE + 16), INVALID),          # workspace not 256-aligned
+    (dict(ws_bytes=100), INVALID),          # workspace too small
+    (dict(flags=1 << 31), INVALID),
+    (dict(Hq=3), INVALID),
+    (dict(w_local=-1), INVALID),
+])
+def test_prefill_3pass_rejects(lib, kw, code):
+    assert _prefill_3pass(lib, **kw) == code
+    assert lib.jl_last_error()
+
+
+def test_prefill_3pass_workspace_size(lib):
+    B, L, Hq, Hkv, D = 1, 1000, 4, 2, 128
+    n = lib.jl_bifocal_prefill_3pass_workspace_size(B, L, Hq, Hkv, D)
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    keys = 2 * up(B * L * Hkv * D * 2)
+    assert n == keys + 2 * up(B * L * Hq * D * 2) + 2 * up(B * Hq * L * 4)
