@@ -203,6 +203,32 @@ jl_status jl_bifocal_decode_noalloc(const void *q_new, const void *k_cache_roped
                                     int w_local, int w_pretrained, double rope_base,
                                     unsigned flags, jl_stream_t stream);
 
+/*
+ * Batched single-token decode, one position per sequence (the batch-size > 1,
+ * ragged case of jl_bifocal_decode; techwalker §三, bittide §3.3).
+ *   pos   HOST array of B positions, 0 <= pos[b] < cache_capacity; sequence b
+ *         decodes its token at pos[b] over cache slots 0..pos[b], with its own
+ *         G = max(1, ceil((pos[b] + 1) / w_pretrained)) and window.
+ *   q_new [B, Hq, D], caches [B, cache_capacity, Hkv, D], out [B, Hq, D],
+ *   lse [B, Hq]: as jl_bifocal_decode.  Cache slots past pos[b] are never
+ *   used (any contents).
+ *   workspace: at least jl_bifocal_decode_batched_workspace_size() bytes,
+ *   256-byte aligned.  The library plans one wave of CTAs over all sequences'
+ *   keys on the host and copies the plan (a few KiB, from pageable memory)
+ *   into the workspace on `stream` before the kernels; the call is therefore
+ *   not capturable in a CUDA graph.
+ *   D == 128, Hkv <= 8, Hq / Hkv <= 8 (JL_ERR_UNSUPPORTED otherwise).
+ *   flags: JL_FLAG_NO_BIFOCAL.
+ */
+size_t jl_bifocal_decode_batched_workspace_size(int B, int Hq, int Hkv, int D);
+jl_status jl_bifocal_decode_batched(const void *q_new, const void *k_cache_roped,
+                                    const void *v_cache, const int *pos,
+                                    int cache_capacity, void *out, float *lse,
+                                    void *workspace, size_t workspace_bytes, int B,
+                                    int Hq, int Hkv, int D, int w_local,
+                                    int w_pretrained, double rope_base,
+                                    unsigned flags, jl_stream_t stream);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 const char *jl_last_error(void);
 

@@ -17,6 +17,7 @@ __all__ = [
     "NO_BIFOCAL", "DEBUG_SKIP_ARRIVE", "JetLongError", "group_size", "bifocal_prefill",
     "prefill_workspace_size", "decode_workspace_size", "bifocal_decode",
     "bifocal_prefill_3pass", "prefill_3pass_workspace_size",
+    "bifocal_decode_batched", "decode_batched_workspace_size",
     "bifocal_decode_noalloc",
     "check_device_status", "finalize", "library_path", "load",
 ]
@@ -73,6 +74,11 @@ def load():
     L.jl_bifocal_decode.restype = i
     L.jl_bifocal_decode.argtypes = [p, p, p, i, i, p, p, p, sz, i, i, i, i, i, i, d,
                                     u, p]
+    L.jl_bifocal_decode_batched_workspace_size.restype = sz
+    L.jl_bifocal_decode_batched_workspace_size.argtypes = [i, i, i, i]
+    L.jl_bifocal_decode_batched.restype = i
+    L.jl_bifocal_decode_batched.argtypes = [p, p, p, p, i, p, p, p, sz, i, i, i, i, i, i, d,
+                                            u, p]
     L.jl_bifocal_decode_noalloc.restype = i
     L.jl_bifocal_decode_noalloc.argtypes = [p, p, p, i, i, p, p, i, i, i, i, i, i, d, u, p]
     L.jl_last_error.restype = ctypes.c_char_p
@@ -216,6 +222,42 @@ def bifocal_decode(q_new, k_cache, v_cache, pos, *, w_local, w_pretrained, rope_
             _ptr(q_new), _ptr(k_cache), _ptr(v_cache), int(pos), cap, _ptr(out),
             _ptr(lse), _ptr(workspace), workspace.numel(), B, Hq, Hkv, D, int(w_local),
             int(w_pretrained), float(rope_base), int(flags), _stream(stream)))
+    return out, lse
+
+
+def decode_batched_workspace_size(B, Hq, Hkv, D) -> int:
+    return int(load().jl_bifocal_decode_batched_workspace_size(B, Hq, Hkv, D))
+
+
+def bifocal_decode_batched(q_new, k_cache, v_cache, pos, *, w_local, w_pretrained, rope_base,
+                           out=None, lse=None, workspace=None, flags=0, stream=None):
+    """Single-token decode of B sequences, sequence b at position pos[b] (a
+    sequence of B ints).  q_new [B,Hq,D] pre-RoPE bf16; caches [B,cap,Hkv,D]
+    bf16 with keys rotated at their original positions.  Returns (out, lse)."""
+    B, Hq, D = q_new.shape
+    cap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _need(q_new, "q_new", torch.bfloat16)
+    _need(k_cache, "k_cache", torch.bfloat16, (B, cap, Hkv, D))
+    _need(v_cache, "v_cache", torch.bfloat16, (B, cap, Hkv, D))
+    pos = [int(x) for x in pos]
+    if len(pos) != B:
+        raise ValueError(f"pos must hold {B} positions, got {len(pos)}")
+    pos_arr = (ctypes.c_int * B)(*pos)
+    if out is None:
+        out = torch.empty_like(q_new)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q_new.device)
+    _need(out, "out", torch.bfloat16, (B, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq))
+    if workspace is None:
+        workspace = torch.empty(max(decode_batched_workspace_size(B, Hq, Hkv, D), 16),
+                                dtype=torch.uint8, device=q_new.device)
+    _need(workspace, "workspace", torch.uint8)
+    with torch.cuda.device(q_new.device):
+        _check(load().jl_bifocal_decode_batched(
+            _ptr(q_new), _ptr(k_cache), _ptr(v_cache), pos_arr, cap, _ptr(out), _ptr(lse),
+            _ptr(workspace), workspace.numel(), B, Hq, Hkv, D, int(w_local), int(w_pretrained),
+            float(rope_base), int(flags), _stream(stream)))
     return out, lse
 
 

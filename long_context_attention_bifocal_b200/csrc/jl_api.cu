@@ -15,6 +15,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "jl_internal.h"
 
@@ -481,6 +482,132 @@ jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped, const 
     e = launch_decode(a, s);
   }
   return e == cudaSuccess ? JL_OK : cuda_fail(e, "decode launch");
+}
+
+size_t jl_bifocal_decode_batched_workspace_size(int B, int Hq, int Hkv, int D) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || D != 128) return 0;
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t n_max = static_cast<size_t>(kDecodeBatchCtas) + 2 * static_cast<size_t>(B);
+  return up(n_max * sizeof(DecodeWork)) + up(static_cast<size_t>(B) * sizeof(DecodeSeq)) +
+         n_max * Hq * kDecodePartialFloats * sizeof(float);
+}
+
+jl_status jl_bifocal_decode_batched(const void *q_new, const void *k_cache_roped,
+                                    const void *v_cache, const int *pos, int cache_capacity,
+                                    void *out, float *lse, void *workspace,
+                                    size_t workspace_bytes, int B, int Hq, int Hkv, int D,
+                                    int w_local, int w_pretrained, double rope_base,
+                                    unsigned flags, jl_stream_t stream) {
+  g_last_error.clear();
+  jl_status st = check_common(B, 1, Hq, Hkv, D, w_local, w_pretrained, rope_base);
+  if (st != JL_OK) return st;
+  if (!q_new || !k_cache_roped || !v_cache || !out || !lse || !workspace || !pos)
+    return fail(JL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q_new) || !aligned16(k_cache_roped) || !aligned16(v_cache) ||
+      !aligned16(out) || !aligned16(lse))
+    return fail(JL_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(JL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL)) != 0)
+    return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if (D != 128) return fail(JL_ERR_UNSUPPORTED, "decode supports head dim 128 (got %d)", D);
+  if (!decode_mma_supported(Hq, Hkv, D))
+    return fail(JL_ERR_UNSUPPORTED,
+                "batched decode needs the tensor-core kernel (Hkv <= 8, Hq / Hkv <= 8)");
+  if (cache_capacity < 1) return fail(JL_ERR_INVALID_ARG, "cache_capacity must be >= 1");
+  long long total = 0;
+  int max_keys = 0;
+  for (int b = 0; b < B; ++b) {
+    if (pos[b] < 0 || pos[b] >= cache_capacity)
+      return fail(JL_ERR_INVALID_ARG, "need 0 <= pos[%d] (%d) < cache_capacity (%d)", b, pos[b],
+                  cache_capacity);
+    total += static_cast<long long>(pos[b]) + 1;
+    max_keys = pos[b] + 1 > max_keys ? pos[b] + 1 : max_keys;
+  }
+  const size_t need = jl_bifocal_decode_batched_workspace_size(B, Hq, Hkv, D);
+  if (workspace_bytes < need)
+    return fail(JL_ERR_INVALID_ARG, "workspace too small: %zu bytes, need %zu", workspace_bytes,
+                need);
+
+  // Plan: one wave of CTAs over all keys; each sequence's remote range
+  // [0, far_end) and local range [far_end, pos] are cut into chunks of at most
+  // `chunk` keys (a multiple of 16), so at most kDecodeBatchCtas + 2B chunks.
+  long long chunk = (total + kDecodeBatchCtas - 1) / kDecodeBatchCtas;
+  chunk = ((chunk + 15) / 16) * 16;
+  if (chunk < 16) chunk = 16;
+  std::vector<DecodeWork> work;
+  std::vector<DecodeSeq> seqs(B);
+  for (int b = 0; b < B; ++b) {
+    const int p = pos[b];
+    const long long G = group_size_ll(static_cast<long long>(p) + 1, w_pretrained);
+    const bool plain = (flags & JL_FLAG_NO_BIFOCAL) || G == 1;
+    const long long fe = static_cast<long long>(p) + 1 - w_local;
+    const int far_end = plain ? 0 : static_cast<int>(fe < 0 ? 0 : fe);
+    const unsigned long long magic =
+        G >= 2 ? (~0ull / static_cast<unsigned long long>(G)) + 1ull : 0ull;
+    seqs[b].first = static_cast<int>(work.size());
+    auto cut = [&](int lo, int hi, int far) {
+      for (long long k0 = lo; k0 < hi; k0 += chunk) {
+        DecodeWork w;
+        w.b = b;
+        w.k_begin = static_cast<int>(k0);
+        w.k_end = static_cast<int>(k0 + chunk < hi ? k0 + chunk : hi);
+        w.far = far;
+        w.pos = p;
+        w.G = static_cast<int>(G);
+        w.part = static_cast<int>(work.size()) * Hq;
+        w.pad = 0;
+        w.g_magic = magic;
+        work.push_back(w);
+      }
+    };
+    cut(0, far_end, 1);
+    cut(far_end, p + 1, 0);
+    seqs[b].n = static_cast<int>(work.size()) - seqs[b].first;
+  }
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t n_max = static_cast<size_t>(kDecodeBatchCtas) + 2 * static_cast<size_t>(B);
+  if (work.size() > n_max) return fail(JL_ERR_CUDA, "internal: decode plan too large");
+  const size_t work_bytes = up(n_max * sizeof(DecodeWork));
+  std::vector<unsigned char> tables(work_bytes + B * sizeof(DecodeSeq));
+  std::memcpy(tables.data(), work.data(), work.size() * sizeof(DecodeWork));
+  std::memcpy(tables.data() + work_bytes, seqs.data(), B * sizeof(DecodeSeq));
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DecodeArgs a;
+  a.q = static_cast<const __nv_bfloat16 *>(q_new);
+  a.kc = static_cast<const __nv_bfloat16 *>(k_cache_roped);
+  a.vc = static_cast<const __nv_bfloat16 *>(v_cache);
+  a.out = static_cast<__nv_bfloat16 *>(out);
+  a.lse = lse;
+  char *ws = static_cast<char *>(workspace);
+  a.work = reinterpret_cast<const DecodeWork *>(ws);
+  a.seqs = reinterpret_cast<const DecodeSeq *>(ws + work_bytes);
+  a.ws = reinterpret_cast<float *>(ws + work_bytes + up(B * sizeof(DecodeSeq)));
+  a.n_work = static_cast<int>(work.size());
+  a.max_keys = max_keys;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.D = D;
+  a.pos = max_keys - 1;
+  a.cap = cache_capacity;
+  a.G = 1;
+  a.far_end = 0;
+  a.chunk = static_cast<int>(chunk);
+  a.n_far_chunks = 0;
+  a.n_chunks = a.n_work;
+  a.scale = static_cast<float>(1.0 / std::sqrt(D));
+  st = rope_table(D, rope_base, max_keys < 64 ? 64 : max_keys, s, &a.table);
+  if (st != JL_OK) return st;
+  unsigned *status = nullptr;
+  st = status_word(&status);
+  if (st != JL_OK) return st;
+  // pageable source: the copy is staged before the call returns
+  cudaError_t e = cudaMemcpyAsync(ws, tables.data(), tables.size(), cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode table copy");
+  e = launch_decode_mma(a, status, s);
+  return e == cudaSuccess ? JL_OK : cuda_fail(e, "batched decode launch");
 }
 
 jl_status jl_bifocal_decode_noalloc(const void *q_new, const void *k_cache_roped,

@@ -332,17 +332,30 @@ constexpr int kCombineSlice = 32;
 constexpr int kCombineSlices = kD / kCombineSlice;
 __global__ void __launch_bounds__(kCombineThreads)
     bifocal_decode_combine_kernel(const float *__restrict__ ws, __nv_bfloat16 *__restrict__ out,
-                                  float *__restrict__ lse, int n_chunks) {
+                                  float *__restrict__ lse, int n_chunks, int Hq,
+                                  const DecodeSeq *__restrict__ seqs) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int kW = kCombineThreads / 32;
   __shared__ float part[kW][kCombineSlice];
   __shared__ float wmax[kW], wsum[kW];
   const int bh = blockIdx.x / kCombineSlices, sl = blockIdx.x % kCombineSlices;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const float *src = ws + static_cast<int64_t>(bh) * n_chunks * kDecodePartialFloats;
+  // chunk c of (batch, head) bh at src + c * stride; one position for every
+  // sequence: [bh][chunk] layout; batched: [chunk][head] from the sequence table
+  const float *src;
+  int64_t stride;
+  if (seqs != nullptr) {
+    const DecodeSeq q = seqs[bh / Hq];
+    n_chunks = q.n;
+    src = ws + (static_cast<int64_t>(q.first) * Hq + bh % Hq) * kDecodePartialFloats;
+    stride = static_cast<int64_t>(Hq) * kDecodePartialFloats;
+  } else {
+    src = ws + static_cast<int64_t>(bh) * n_chunks * kDecodePartialFloats;
+    stride = kDecodePartialFloats;
+  }
   float mx = -INFINITY;
   for (int c = t; c < n_chunks; c += kCombineThreads)
-    mx = fmaxf(mx, src[c * kDecodePartialFloats + kD]);
+    mx = fmaxf(mx, src[c * stride + kD]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   if (lane == 0) wmax[warp] = mx;
@@ -353,7 +366,7 @@ __global__ void __launch_bounds__(kCombineThreads)
   float acc = 0.f, lsum = 0.f;
 #pragma unroll 4
   for (int c = warp; c < n_chunks; c += kW) {
-    const float *pc = src + static_cast<int64_t>(c) * kDecodePartialFloats;
+    const float *pc = src + static_cast<int64_t>(c) * stride;
     const float mc = pc[kD];
     const float f = (mc == -INFINITY) ? 0.f : ex2(mc - M);
     acc = fmaf(f, pc[kCombineSlice * sl + lane], acc);
@@ -463,7 +476,7 @@ cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t s) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, bifocal_decode_combine_kernel, static_cast<const float *>(a.ws),
-                            a.out, a.lse, a.n_chunks);
+                            a.out, a.lse, a.n_chunks, a.Hq, a.seqs);
 }
 
 size_t decode_ws_floats(int B, int Hq, int D, int n_chunks) {

@@ -80,6 +80,7 @@ struct Params {
   float scale_log2;
   unsigned long long g_magic;  // ceil(2^64 / G): floor(k / G) = umulhi(k, g_magic), G >= 2
   int skip_first_arrival;  // test-only: withhold the first block (bounded-wait check)
+  const DecodeWork *work;  // batched decode: this CTA's entry (nullptr: one position for all)
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1,
@@ -154,15 +155,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.x, b = blockIdx.y;
-  const bool far = c < p.n_far;
-  int k_begin, k_end;
-  if (far) {
-    k_begin = c * p.chunk;
-    k_end = min(p.far_end, k_begin + p.chunk);
+  // this CTA's keys [k_begin, k_end) of sequence b, and where its partials go:
+  // query head h of the chunk at (pbase + h * pstride) * kDecodePartialFloats
+  int b, k_begin, k_end, pos, G;
+  bool far;
+  unsigned long long g_magic;
+  int64_t pbase, pstride;
+  if (p.work != nullptr) {  // batched: one entry of the host-planned work table
+    const DecodeWork w = p.work[blockIdx.x];
+    b = w.b;
+    k_begin = w.k_begin;
+    k_end = w.k_end;
+    far = w.far != 0;
+    pos = w.pos;
+    G = w.G;
+    g_magic = w.g_magic;
+    pbase = w.part;
+    pstride = 1;
   } else {
-    k_begin = p.far_end + (c - p.n_far) * p.chunk;
-    k_end = min(p.pos + 1, k_begin + p.chunk);
+    const int c = blockIdx.x;
+    b = blockIdx.y;
+    far = c < p.n_far;
+    if (far) {
+      k_begin = c * p.chunk;
+      k_end = min(p.far_end, k_begin + p.chunk);
+    } else {
+      k_begin = p.far_end + (c - p.n_far) * p.chunk;
+      k_end = min(p.pos + 1, k_begin + p.chunk);
+    }
+    pos = p.pos;
+    G = p.G;
+    g_magic = p.g_magic;
+    pbase = static_cast<int64_t>(b) * p.Hq * p.n_chunks + c;
+    pstride = p.n_chunks;
   }
   const int nblk = (k_end - k_begin + kBlock - 1) / kBlock;
 
@@ -240,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float4 step[kBlock];
 #pragma unroll
     for (int r = 0; r < kBlock; ++r) step[r] = cs4[r * (kHalf / 2) + lane];
-    int u0 = k_begin - div_g(k_begin, p.g_magic);
+    int u0 = k_begin - div_g(k_begin, g_magic);
     float4 base = cs4[static_cast<int64_t>(u0) * (kHalf / 2) + lane];
     for (int blk = 0; blk < nblk; ++blk) {
       const int s = blk % kStages;
@@ -255,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float4 cb = base;
       if (blk + 1 < nblk) {
         const int kn = k_begin + (blk + 1) * kBlock;
-        u0 = kn - div_g(kn, p.g_magic);
+        u0 = kn - div_g(kn, g_magic);
         base = cs4[static_cast<int64_t>(u0) * (kHalf / 2) + lane];
       }
       // row r, 8-byte word lane ^ (4 (r % 4)): (c0, c1 | s0, s1) as bf16x2
@@ -287,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Q^T fragments: qb[ks][hh] = head g, dims 16ks + 2cq + 8hh + {0,1}
   uint32_t qb[8][2];
   {
-    const int udq = p.pos - p.pos / p.G;
+    const int udq = pos - pos / G;
     const bool real = g < heads;
     const __nv_bfloat16 *src =
         p.q + (static_cast<int64_t>(b) * p.Hq + hk * p.group + (real ? g : 0)) * kD;
@@ -302,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int i = d0 + e;  // rotation pair (i, i + 64)
           const float x1 = real ? __bfloat162float(src[i]) : 0.f;
           const float x2 = real ? __bfloat162float(src[i + kHalf]) : 0.f;
-          const float2 a = p.cs[static_cast<int64_t>(p.pos) * kHalf + i];
+          const float2 a = p.cs[static_cast<int64_t>(pos) * kHalf + i];
           float z1 = x1 * a.x - x2 * a.y;
           float z2 = x1 * a.y + x2 * a.x;
           if (far) {  // by dq = -udq
@@ -361,11 +386,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // pp ^ (4 (row % 4)) as (c0, c1 | s0, s1), bf16x2 (conflict-free: the
       // keys of a half-warp fall on at most 4 consecutive rows)
       const uint8_t *tab = smem + s * kStageBytes + 2 * kKBytes;
-      const int u0 = k0 - div_g(k0, p.g_magic);
+      const int u0 = k0 - div_g(k0, g_magic);
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int kk = k0 + g + 8 * r;
-        const int urow = (kk - div_g(kk, p.g_magic)) - u0;  // 0..15
+        const int urow = (kk - div_g(kk, g_magic)) - u0;  // 0..15
         const uint8_t *trow = tab + urow * kTabRow;
         const int sw = (urow & 3) << 2;
 #pragma unroll
@@ -386,6 +411,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int mt = 0; mt < 8; ++mt)
       ldsm_x4_t(vt + tile_off(vrow, 2 * mt + ((lane >> 3) & 1)), vf[mt][0], vf[mt][1], vf[mt][2],
                 vf[mt][3]);
+    if (k0 + kBlock > k_end) {
+      // keys past the chunk's end: their P is 0, and their V (possibly past a
+      // sequence's last key, so any value) must not reach O as 0 * inf or NaN
+      const uint32_t m0 = (k0 + 2 * cq < k_end ? 0x0000FFFFu : 0u) |
+                          (k0 + 2 * cq + 1 < k_end ? 0xFFFF0000u : 0u);
+      const uint32_t m1 = (k0 + 8 + 2 * cq < k_end ? 0x0000FFFFu : 0u) |
+                          (k0 + 9 + 2 * cq < k_end ? 0xFFFF0000u : 0u);
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        vf[mt][0] &= m0;
+        vf[mt][1] &= m0;
+        vf[mt][2] &= m1;
+        vf[mt][3] &= m1;
+      }
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(bar(kStages + s));
     // S = K . Q^T, two accumulation chains
@@ -459,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int e = 0; e < 2; ++e) {
     const int h = 2 * cq + e;
     if (h >= heads) continue;
-    float *dst = p.ws + ((static_cast<int64_t>(b) * p.Hq + hk * p.group + h) * p.n_chunks + c) *
+    float *dst = p.ws + (pbase + static_cast<int64_t>(hk * p.group + h) * pstride) *
                             kDecodePartialFloats;
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
@@ -534,9 +574,11 @@ cudaError_t launch_decode_mma(const DecodeArgs &a, unsigned *status, cudaStream_
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   });
   if (attr_err != cudaSuccess) return attr_err;
+  // the maps end at the last valid key (of the longest sequence when batched)
+  const int keys = a.work != nullptr ? a.max_keys : a.pos + 1;
   CUtensorMap mk, mv;
-  if (!make_cache_map(&mk, a.kc, a.B, a.cap, a.pos + 1, a.Hkv) ||
-      !make_cache_map(&mv, a.vc, a.B, a.cap, a.pos + 1, a.Hkv))
+  if (!make_cache_map(&mk, a.kc, a.B, a.cap, keys, a.Hkv) ||
+      !make_cache_map(&mv, a.vc, a.B, a.cap, keys, a.Hkv))
     return cudaErrorInvalidValue;
   Params p;
   p.q = a.q;
@@ -555,7 +597,8 @@ cudaError_t launch_decode_mma(const DecodeArgs &a, unsigned *status, cudaStream_
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.skip_first_arrival = a.debug_skip_arrival ? 1 : 0;
   p.g_magic = a.G >= 2 ? (~0ull / static_cast<unsigned long long>(a.G)) + 1ull : 0ull;
-  dim3 grid(a.n_chunks, a.B);
+  p.work = a.work;
+  const dim3 grid = a.work != nullptr ? dim3(a.n_work) : dim3(a.n_chunks, a.B);
   bifocal_decode_mma_kernel<<<grid, kThreads, kSmemAlloc, s>>>(mk, mv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -68,6 +68,22 @@ bool prefill_x2_supported(const PrefillArgs &a);
 cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_f32(const PrefillArgs &a, cudaStream_t s);
 
+// Batched decode with one position per sequence: the host plans one wave of
+// CTAs over all sequences' keys and copies these tables into the workspace.
+struct DecodeWork {              // one CTA: a key range of one sequence
+  int b;                         // sequence
+  int k_begin, k_end;            // keys [k_begin, k_end), all remote or all local
+  int far;                       // 1: remote keys (corrected)
+  int pos, G;                    // the sequence's position and group size
+  int part;                      // partials of query head h at (part + h) * kDecodePartialFloats
+  int pad;
+  unsigned long long g_magic;    // ceil(2^64 / G) when G >= 2
+};
+struct DecodeSeq {               // one sequence's partials: chunks first .. first + n - 1
+  int first, n;
+};
+constexpr int kDecodeBatchCtas = 148;  // CTAs the batched plan aims for (one B200 wave)
+
 struct DecodeArgs {
   const __nv_bfloat16 *q;   // [B,Hq,D] pre-RoPE
   const __nv_bfloat16 *kc;  // [B,cap,Hkv,D] rotated at original positions
@@ -83,7 +99,13 @@ struct DecodeArgs {
   int chunk;                // keys per split
   int n_far_chunks, n_chunks;
   bool debug_skip_arrival = false;  // JL_FLAG_DEBUG_SKIP_ARRIVE (tensor-core kernel)
+  // batched decode (tensor-core kernel): work table, sequence table, their
+  // sizes, and the largest number of valid keys of any sequence
+  const DecodeWork *work = nullptr;
+  const DecodeSeq *seqs = nullptr;
+  int n_work = 0, max_keys = 0;
 };
+
 
 // One split partial in the decode workspace: o[128], m (log2 units), l, and
 // two floats of padding so every partial starts on a 16-byte boundary.

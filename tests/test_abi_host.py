@@ -162,3 +162,38 @@ def test_prefill_3pass_workspace_size(lib):
     up = lambda x: (x + 255) // 256 * 256  # noqa: E731
     keys = 2 * up(B * L * Hkv * D * 2)
     assert n == keys + 2 * up(B * L * Hq * D * 2) + 2 * up(B * Hq * L * 4)
+
+
+def _decode_batched(lib, pos=(100, 5), **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, cap=200, out=FAKE, lse=FAKE, ws=FAKE,
+             ws_bytes=1 << 30, B=len(pos) if pos else 2, Hq=8, Hkv=2, D=128, w_local=16,
+             w_pretrained=64,
+             base=1e6, flags=0)
+    a.update(kw)
+    arr = (ctypes.c_int * len(pos))(*pos) if pos is not None else None
+    return lib.jl_bifocal_decode_batched(a["q"], a["kc"], a["vc"], arr, a["cap"], a["out"],
+                                         a["lse"], a["ws"], a["ws_bytes"], a["B"], a["Hq"],
+                                         a["Hkv"], a["D"], a["w_local"], a["w_pretrained"],
+                                         a["base"], a["flags"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(pos=(100, 200)), INVALID),          # pos >= cap
+    (dict(pos=(100, -1)), INVALID),
+    (dict(pos=None, B=2), INVALID),
+    (dict(D=64), UNSUPPORTED),
+    (dict(Hq=18, Hkv=2), UNSUPPORTED),        # group 9: no tensor-core kernel
+    (dict(ws_bytes=64), INVALID),
+    (dict(ws=FAKE + 16), INVALID),            # not 256-aligned
+    (dict(flags=1 << 31), INVALID),
+])
+def test_decode_batched_rejects(lib, kw, code):
+    pos = kw.pop("pos", (100, 5))
+    assert _decode_batched(lib, pos=pos, **kw) == code
+    assert lib.jl_last_error()
+
+
+def test_decode_batched_workspace_size(lib):
+    n = lib.jl_bifocal_decode_batched_workspace_size(4, 32, 8, 128)
+    assert n >= (148 + 8) * 32 * 132 * 4
+    assert lib.jl_bifocal_decode_batched_workspace_size(4, 32, 8, 64) == 0
