@@ -257,6 +257,26 @@ def run_cuda(args):
         return med(ea), med(eb)
 
     dec_bif, dec_plain = interleaved_ms(lambda: decode(0), lambda: decode(jl.NO_BIFOCAL), 100)
+
+    # a ragged batch: 8 sequences of one shape at different positions (G 1-4)
+    bpos = [16383, 32767, 49151, 65535, 81919, 98303, 114687, 131071]
+    bcap = max(bpos) + 1
+    gb = torch.Generator(device=dev)
+    gb.manual_seed(rank_seed(dc["seed"] + 1, rank))
+    qb = torch.randn((len(bpos), dc["Hq"], dc["D"]), generator=gb, device=dev).to(torch.bfloat16)
+    kb = torch.randn((len(bpos), bcap, dc["Hkv"], dc["D"]), generator=gb,
+                     device=dev).to(torch.bfloat16)
+    vb = torch.randn((len(bpos), bcap, dc["Hkv"], dc["D"]), generator=gb,
+                     device=dev).to(torch.bfloat16)
+    wsb = torch.empty(jl.decode_batched_workspace_size(len(bpos), dc["Hq"], dc["Hkv"], dc["D"]),
+                      dtype=torch.uint8, device=dev)
+    outb = torch.empty_like(qb)
+    lseb = torch.empty((len(bpos), dc["Hq"]), dtype=torch.float32, device=dev)
+    dec_batched = avg_ms(lambda: jl.bifocal_decode_batched(qb, kb, vb, bpos, out=outb, lse=lseb,
+                                                           workspace=wsb, **kwd), 20)
+    batched_bytes = sum(kv_bytes(1, dc["Hkv"], dc["D"], p_ + 1) for p_ in bpos)
+    dec_batched = max_over_ranks(dec_batched, world)
+    del qb, kb, vb, wsb, outb, lseb
     pre_plain = avg_ms(lambda: prefill(jl.NO_BIFOCAL), max(1, min(3, args.steps)))
     pre_bif = avg_ms(lambda: prefill(0), max(1, min(3, args.steps)))
     # the pages' unfused three-call formulation of the same prefill (A + B - C)
@@ -334,6 +354,13 @@ def run_cuda(args):
             "us_per_call_in_step": round(dec_sum / args.steps * 1e3, 2),
             "frac_hbm": round(dec_gbs / world / hbm, 4),
             "overhead_vs_no_bifocal": round(dec_bif / dec_plain - 1.0, 4),
+        },
+        "decode_batched": {
+            "B": len(bpos), "positions": bpos, "inputs": "N(0,1) bf16 on the device, seeded",
+            "us_per_call": round(dec_batched * 1e3, 2),
+            "value": round(batched_bytes * world / (dec_batched / 1e3) / 1e9, 1),
+            "unit": "GB/s",
+            "frac_hbm": round(batched_bytes / (dec_batched / 1e3) / 1e9 / hbm, 4),
         },
         "prefill_unfused_3pass": {
             "ms_per_call": round(pre_3pass, 3),

@@ -145,6 +145,37 @@ jl_status jl_bifocal_prefill_3pass(const void *q, const void *k, const void *v,
                                    void *workspace, size_t workspace_bytes,
                                    jl_stream_t stream);
 
+/*
+ * Chunked prefill against a cache: Lq new tokens attend to a cached prefix and
+ * to themselves (a long prompt processed in pieces, or text appended to a long
+ * context; techwalker §三 for the cache at original positions).
+ *   q              [B, Lq, Hq, D] bf16, pre-RoPE; row r is the token at position
+ *                  q_offset + r
+ *   k_cache_roped  [B, cache_capacity, Hkv, D] bf16, keys rotated by standard
+ *                  RoPE at their original positions (the decode cache layout);
+ *                  slots 0 .. q_offset + Lq - 1 valid (the prefix and this
+ *                  chunk, written by the caller)
+ *   v_cache        [B, cache_capacity, Hkv, D] bf16, the same slots valid
+ *   out [B, Lq, Hq, D] bf16 and lse [B, Hq, Lq] fp32 (written)
+ * G = max(1, ceil((q_offset + Lq) / w_pretrained)) from the total length, and
+ * the local/remote rule of jl_bifocal_prefill over keys [0, q_offset + Lq): the
+ * result is rows q_offset .. q_offset + Lq - 1 of jl_bifocal_prefill over the
+ * whole sequence (up to the bf16 rounding of the cached keys).  Keys at
+ * remapped positions are formed from the cache as R(f(k) - k) k_cache.
+ * q_offset a multiple of 128 (JL_ERR_UNSUPPORTED otherwise), q_offset + Lq <=
+ * cache_capacity, D == 128, flags: JL_FLAG_NO_BIFOCAL.
+ * workspace: at least jl_bifocal_prefill_chunk_workspace_size() bytes,
+ * 256-byte aligned (the remapped keys); NULL selects the library's scratch.
+ */
+size_t jl_bifocal_prefill_chunk_workspace_size(int B, int q_offset, int Lq, int Hkv,
+                                               int D);
+jl_status jl_bifocal_prefill_chunk(const void *q, const void *k_cache_roped,
+                                   const void *v_cache, int q_offset, int cache_capacity,
+                                   void *out, float *lse, int B, int Lq, int Hq, int Hkv,
+                                   int D, int w_local, int w_pretrained, double rope_base,
+                                   unsigned flags, void *workspace, size_t workspace_bytes,
+                                   jl_stream_t stream);
+
 /* Bytes of workspace jl_bifocal_decode needs for these sizes. */
 size_t jl_bifocal_decode_workspace_size(int B, int Hq, int Hkv, int D, int pos);
 

@@ -18,6 +18,7 @@ __all__ = [
     "prefill_workspace_size", "decode_workspace_size", "bifocal_decode",
     "bifocal_prefill_3pass", "prefill_3pass_workspace_size",
     "bifocal_decode_batched", "decode_batched_workspace_size",
+    "bifocal_prefill_chunk", "prefill_chunk_workspace_size",
     "bifocal_decode_noalloc",
     "check_device_status", "finalize", "library_path", "load",
 ]
@@ -69,6 +70,11 @@ def load():
     L.jl_bifocal_prefill_3pass_workspace_size.argtypes = [i, i, i, i, i]
     L.jl_bifocal_prefill_3pass.restype = i
     L.jl_bifocal_prefill_3pass.argtypes = [p, p, p, p, p, i, i, i, i, i, i, i, d, u, p, sz, p]
+    L.jl_bifocal_prefill_chunk_workspace_size.restype = sz
+    L.jl_bifocal_prefill_chunk_workspace_size.argtypes = [i, i, i, i, i]
+    L.jl_bifocal_prefill_chunk.restype = i
+    L.jl_bifocal_prefill_chunk.argtypes = [p, p, p, i, i, p, p, i, i, i, i, i, i, i, d, u, p,
+                                           sz, p]
     L.jl_bifocal_decode_workspace_size.restype = sz
     L.jl_bifocal_decode_workspace_size.argtypes = [i, i, i, i, i]
     L.jl_bifocal_decode.restype = i
@@ -190,6 +196,38 @@ def bifocal_prefill_3pass(q, k, v, *, w_local, w_pretrained, rope_base, out=None
             _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, L, Hq, Hkv, D, int(w_local),
             int(w_pretrained), float(rope_base), int(flags), _ptr(workspace),
             workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def prefill_chunk_workspace_size(B, q_offset, Lq, Hkv, D) -> int:
+    return int(load().jl_bifocal_prefill_chunk_workspace_size(B, q_offset, Lq, Hkv, D))
+
+
+def bifocal_prefill_chunk(q, k_cache, v_cache, q_offset, *, w_local, w_pretrained, rope_base,
+                          out=None, lse=None, flags=0, workspace=None, stream=None):
+    """Chunked prefill: q [B,Lq,Hq,D] pre-RoPE bf16 at positions q_offset + r
+    against caches [B,cap,Hkv,D] bf16 (keys rotated at original positions,
+    slots 0..q_offset+Lq-1 valid).  Returns (out [B,Lq,Hq,D], lse [B,Hq,Lq])."""
+    B, Lq, Hq, D = q.shape
+    cap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _need(q, "q", torch.bfloat16)
+    _need(k_cache, "k_cache", torch.bfloat16, (B, cap, Hkv, D))
+    _need(v_cache, "v_cache", torch.bfloat16, (B, cap, Hkv, D))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.bfloat16, (B, Lq, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq, Lq))
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8)
+        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel()
+    with torch.cuda.device(q.device):
+        _check(load().jl_bifocal_prefill_chunk(
+            _ptr(q), _ptr(k_cache), _ptr(v_cache), int(q_offset), cap, _ptr(out), _ptr(lse), B,
+            Lq, Hq, Hkv, D, int(w_local), int(w_pretrained), float(rope_base), int(flags),
+            ws_ptr, ws_bytes, _stream(stream)))
     return out, lse
 
 

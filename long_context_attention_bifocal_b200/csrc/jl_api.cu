@@ -312,6 +312,90 @@ jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v, void *
                                rope_base, JL_BF16, 0.f, 0u, nullptr, 0, stream);
 }
 
+size_t jl_bifocal_prefill_chunk_workspace_size(int B, int q_offset, int Lq, int Hkv, int D) {
+  if (B < 1 || q_offset < 0 || Lq < 1 || Hkv < 1 || D < 2) return 0;
+  const size_t one =
+      static_cast<size_t>(B) * (static_cast<size_t>(q_offset) + Lq) * Hkv * D * sizeof(__nv_bfloat16);
+  return (one + 255) & ~static_cast<size_t>(255);
+}
+
+jl_status jl_bifocal_prefill_chunk(const void *q, const void *k_cache_roped, const void *v_cache,
+                                   int q_offset, int cache_capacity, void *out, float *lse, int B,
+                                   int Lq, int Hq, int Hkv, int D, int w_local, int w_pretrained,
+                                   double rope_base, unsigned flags, void *workspace,
+                                   size_t workspace_bytes, jl_stream_t stream) {
+  g_last_error.clear();
+  jl_status st = check_common(B, Lq, Hq, Hkv, D, w_local, w_pretrained, rope_base);
+  if (st != JL_OK) return st;
+  if (!q || !k_cache_roped || !v_cache || !out || !lse)
+    return fail(JL_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k_cache_roped) || !aligned16(v_cache) || !aligned16(out) ||
+      !aligned16(lse))
+    return fail(JL_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL)) != 0)
+    return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if (D != 128) return fail(JL_ERR_UNSUPPORTED, "chunked prefill supports head dim 128 (got %d)", D);
+  if (q_offset < 0 || q_offset % 128 != 0)
+    return fail(JL_ERR_UNSUPPORTED, "q_offset (%d) must be a non-negative multiple of 128",
+                q_offset);
+  const long long Lk = static_cast<long long>(q_offset) + Lq;
+  if (Lk > cache_capacity)
+    return fail(JL_ERR_INVALID_ARG, "q_offset + Lq (%lld) exceeds cache_capacity (%d)", Lk,
+                cache_capacity);
+  if (Lk >= (1LL << 31) - 256) return fail(JL_ERR_UNSUPPORTED, "sequence too long");
+  if (static_cast<long long>((Lq + 127) / 128) * B * Hq >= (1LL << 31))
+    return fail(JL_ERR_UNSUPPORTED, "problem too large for one launch");
+  const size_t need = jl_bifocal_prefill_chunk_workspace_size(B, q_offset, Lq, Hkv, D);
+  if (workspace != nullptr) {
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return fail(JL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (workspace_bytes < need)
+      return fail(JL_ERR_INVALID_ARG, "workspace too small: %zu bytes, need %zu",
+                  workspace_bytes, need);
+  }
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long G = group_size_ll(Lk, w_pretrained);
+  const bool plain = (flags & JL_FLAG_NO_BIFOCAL) || G == 1 || w_local >= Lk;
+  PrefillArgs a;
+  a.q = q;
+  a.v = v_cache;
+  a.out = out;
+  a.lse = lse;
+  a.B = B;
+  a.L = Lq;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.D = D;
+  a.G = static_cast<int>(G);
+  a.w_eff = plain ? INT_MAX : w_local;
+  a.scale = static_cast<float>(1.0 / std::sqrt(D));
+  a.q_off = q_offset;
+  a.kv_stride = cache_capacity;
+  st = rope_table(D, rope_base, static_cast<int>(Lk), s, &a.table);
+  if (st != JL_OK) return st;
+  st = status_word(&a.status);
+  if (st != JL_OK) return st;
+  // keys at original positions: the cache itself; at remapped positions: a
+  // compact corrected copy in the workspace
+  a.kstd = a.w_eff > 0 ? k_cache_roped : nullptr;
+  a.krem = nullptr;
+  if (!plain) {
+    void *ws = workspace;
+    if (ws == nullptr) {
+      st = prefill_scratch(need, &ws);
+      if (st != JL_OK) return st;
+    }
+    cudaError_t e = launch_correct_keys(static_cast<const __nv_bfloat16 *>(k_cache_roped),
+                                        static_cast<__nv_bfloat16 *>(ws), a.table, B,
+                                        static_cast<int>(Lk), cache_capacity, Hkv, D, a.G, s);
+    if (e != cudaSuccess) return cuda_fail(e, "key correction launch");
+    a.krem = ws;
+  }
+  cudaError_t e = launch_attention(a, s);
+  return e == cudaSuccess ? JL_OK : cuda_fail(e, "chunked prefill launch");
+}
+
 size_t jl_bifocal_prefill_3pass_workspace_size(int B, int L, int Hq, int Hkv, int D) {
   if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || D < 2) return 0;
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };

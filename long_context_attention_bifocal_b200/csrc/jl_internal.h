@@ -39,6 +39,12 @@ int sm_count();
 // ---- launchers (each returns the launch's cudaError_t) ----
 cudaError_t launch_rope_table(float2 *cs, int positions, int D, double base, cudaStream_t s);
 
+// Keys [0, L) of a cache [B, cap, Hkv, D] rotated at their original positions,
+// moved to remapped positions: krem[b, k] = R(f(k) - k) kc[b, k], written
+// compactly as [B, L, Hkv, D].
+cudaError_t launch_correct_keys(const __nv_bfloat16 *kc, __nv_bfloat16 *krem, RopeTable t,
+                                int B, int L, int cap, int Hkv, int D, int G, cudaStream_t s);
+
 // Rotated copies of the keys of a [B,L,Hkv,D] bf16 tensor:
 // kstd = R(l) k (if kstd), krem = R(floor(l/G)) k (if krem).
 cudaError_t launch_rotate_keys(const __nv_bfloat16 *k, __nv_bfloat16 *kstd,
@@ -60,6 +66,8 @@ struct PrefillArgs {
   RopeTable table;
   unsigned *status;
   int band = 0;       // 0: bifocal rule; 1 / 2: only the local window, standard / remapped
+  int q_off = 0;      // position of query row 0 (multiple of 128); keys are [0, q_off + L)
+  int64_t kv_stride = 0;  // keys per batch entry in v (and a cache-resident kstd); 0: q_off + L
 };
 
 cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s);

@@ -100,7 +100,8 @@ struct KParams {
   const float2 *cs;
   unsigned *status;
   int B, L, Hq, Hkv, G, w, n_qtiles;
-  int band;  // kBandNone, kBandStd or kBandRem
+  int band;   // kBandNone, kBandStd or kBandRem
+  int q_off;  // position of query row 0 (a multiple of 128; keys start at 0)
   float scale_log2;  // softmax scale * log2(e)
 };
 
@@ -159,11 +160,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < 4) {
       // ------------------------------------------------ softmax warpgroup --
       const int r = threadIdx.x;  // query row within the tile == TMEM lane
-      const int qpos = kBM * qt + r;
-      const bool row_ok = qpos < p.L;
+      const int row_i = kBM * qt + r;    // row of the q / out / lse tensors
+      const int qpos = p.q_off + row_i;  // its position
+      const bool row_ok = row_i < p.L;
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
       const __nv_bfloat16 *qrow =
-          p.q + ((static_cast<int64_t>(b) * p.L + (row_ok ? qpos : 0)) * p.Hq + hq) * kHD;
+          p.q + ((static_cast<int64_t>(b) * p.L + (row_ok ? row_i : 0)) * p.Hq + hq) * kHD;
       const int pos_std = row_ok ? qpos : 0;
       const int pos_rem = row_ok ? qpos / p.G : 0;
       // Q rotated at `pos`, bf16, in the swizzled K-major layout the UMMA
@@ -199,13 +201,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       {
         PassIter t0;
-        t0.begin(qt, p.w, p.band);
+        t0.begin(qt + p.q_off / kBM, p.w, p.band);
         rotate_q(t0.kind() == kRem ? pos_rem : pos_std);
       }
 
       float m = -INFINITY, l = 0.f;
       PassIter t;
-      t.begin(qt, p.w, p.band);
+      t.begin(qt + p.q_off / kBM, p.w, p.band);
       int it = 0;
       bool ok = true;
       while (!t.done()) {
@@ -223,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         const int k0 = kBN * t.j;
         const int mk = t.mask();
-        const bool causal = (t.j == qt);
+        const bool causal = (t.j == qt + p.q_off / kBM);
         const int kind = t.kind();
         t.next();
         if (kind == kRem && !t.done() && t.kind() == kStd)
@@ -342,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const float inv = 1.f / l;
         __nv_bfloat16 *orow =
-            p.out + ((static_cast<int64_t>(b) * p.L + (row_ok ? qpos : 0)) * p.Hq + hq) * kHD;
+            p.out + ((static_cast<int64_t>(b) * p.L + (row_ok ? row_i : 0)) * p.Hq + hq) * kHD;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float o[32];
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (row_ok)
-          p.lse[(static_cast<int64_t>(b) * p.Hq + hq) * p.L + qpos] =
+          p.lse[(static_cast<int64_t>(b) * p.Hq + hq) * p.L + row_i] =
               (m + __log2f(l)) * 0.69314718055994530942f;
       }
     } else if (warp == 4) {
@@ -370,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_krem);
         prefetch_tmap(&tm_v);
         PassIter t;
-        t.begin(qt, p.w, p.band);
+        t.begin(qt + p.q_off / kBM, p.w, p.band);
         int kiss = 0, viss = 0;  // loads issued
         while (!t.done()) {
           const int s = kiss % kStages;
@@ -430,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         PassIter t;
-        t.begin(qt, p.w, p.band);
+        t.begin(qt + p.q_off / kBM, p.w, p.band);
         int it = 0, qphase = 0, prev_kind = t.kind();
         while (ok && !t.done()) {
           const int kind = t.kind();
@@ -501,14 +503,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // [B, L, H, 128] bf16 -> 4-D map (dims innermost first: D, H, L, B), box of
 // 64 dims x 1 head x 128 rows, 128-byte swizzle, zero fill out of bounds.
-bool make_map(CUtensorMap *m, const void *base, int B, int L, int H) {
+bool make_map(CUtensorMap *m, const void *base, int B, int L, int H, int64_t stride_L = 0) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHD), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHD) * 2,
                                  static_cast<cuuint64_t>(H) * kHD * 2,
-                                 static_cast<cuuint64_t>(L) * H * kHD * 2};
+                                 static_cast<cuuint64_t>(stride_L > 0 ? stride_L : L) * H * kHD * 2};
   const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBN), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
@@ -530,8 +532,13 @@ cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s) {
   CUtensorMap mks, mkr, mv;
   const void *krem = a.krem ? a.krem : a.kstd;
   const void *kstd = a.kstd ? a.kstd : a.krem;
-  if (!make_map(&mks, kstd, a.B, a.L, a.Hkv) || !make_map(&mkr, krem, a.B, a.L, a.Hkv) ||
-      !make_map(&mv, a.v, a.B, a.L, a.Hkv))
+  // keys [0, q_off + L); the cache-resident tensors (K_std, V) may be longer
+  // per batch entry than that (kv_stride keys)
+  const int keys = a.q_off + a.L;
+  const int64_t kvs = a.kv_stride > 0 ? a.kv_stride : keys;
+  if (!make_map(&mks, kstd, a.B, keys, a.Hkv, a.kstd ? kvs : keys) ||
+      !make_map(&mkr, krem, a.B, keys, a.Hkv, a.krem ? keys : kvs) ||
+      !make_map(&mv, a.v, a.B, keys, a.Hkv, kvs))
     return cudaErrorInvalidValue;
   KParams p;
   p.q = static_cast<const __nv_bfloat16 *>(a.q);
@@ -546,6 +553,7 @@ cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s) {
   p.G = a.G;
   p.w = a.w_eff;
   p.band = a.band;
+  p.q_off = a.q_off;
   p.n_qtiles = (a.L + kBM - 1) / kBM;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * a.Hq;

@@ -99,7 +99,8 @@ struct KParams {
   const float2 *cs;
   unsigned *status;
   int B, L, Hq, Hkv, G, w, n_qtiles;
-  int band;  // kBandNone, kBandStd or kBandRem
+  int band;   // kBandNone, kBandStd or kBandRem
+  int q_off;  // position of query row 0 (a multiple of 128; keys start at 0)
   float scale_log2;
 };
 
@@ -190,19 +191,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = warp >> 2;           // head of this warpgroup
       const int r = threadIdx.x & 127;   // query row == TMEM lane
       const int hq = hq0 + t;
-      const int qpos = kBM * qt + r;
-      const bool row_ok = qpos < p.L;
+      const int row_i = kBM * qt + r;    // row of the q / out / lse tensors
+      const int qpos = p.q_off + row_i;  // its position
+      const bool row_ok = row_i < p.L;
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
       const uint32_t s_col = lane_base + tm_s(t);
       const uint32_t o_col = lane_base + tm_o(t);
       uint8_t *qdst = smem + (t == 0 ? kOffQ0 : kOffQ1);
       const __nv_bfloat16 *qrow =
-          p.q + ((static_cast<int64_t>(b) * p.L + (row_ok ? qpos : 0)) * p.Hq + hq) * kHD;
+          p.q + ((static_cast<int64_t>(b) * p.L + (row_ok ? row_i : 0)) * p.Hq + hq) * kHD;
       const int pos_std = row_ok ? qpos : 0;
       const int pos_rem = row_ok ? qpos / p.G : 0;
 
       PassIter it;
-      it.begin(qt, p.w, p.band);
+      it.begin(qt + p.q_off / kBM, p.w, p.band);
       // first Q variant = the class of the first pass
       rotate_q_row(qdst, r, qrow, row_ok, p.cs, it.kind() == kRem ? pos_rem : pos_std);
       fence_proxy_async_smem();
@@ -229,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bar(kBarQReady + t));
         }
 
-        const bool causal = (kj == qt);
+        const bool causal = (kj == qt + p.q_off / kBM);
         const bool plain = !causal && mk == kMaskNone;
         const int k0 = kBN * kj;
         // validity of column e for this row (only asked on masked tiles)
@@ -340,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const float inv = 1.f / l;
         __nv_bfloat16 *orow =
-            p.out + ((static_cast<int64_t>(b) * p.L + (row_ok ? qpos : 0)) * p.Hq + hq) * kHD;
+            p.out + ((static_cast<int64_t>(b) * p.L + (row_ok ? row_i : 0)) * p.Hq + hq) * kHD;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float o[32];
@@ -358,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (row_ok)
-          p.lse[(static_cast<int64_t>(b) * p.Hq + hq) * p.L + qpos] =
+          p.lse[(static_cast<int64_t>(b) * p.Hq + hq) * p.L + row_i] =
               (m + __log2f(l)) * 0.69314718055994530942f;
       }
     } else if (warp == kProducerWarp) {
@@ -368,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_krem);
         prefetch_tmap(&tm_v);
         PassIter it;
-        it.begin(qt, p.w, p.band);
+        it.begin(qt + p.q_off / kBM, p.w, p.band);
         int kiss = 0, viss = 0;
         while (!it.done()) {
           const int s = kiss % kStages;
@@ -415,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // PV_t(j), which has read them.  While head t's softmax runs on S_t(j),
         // the tensor core works on head 1-t.
         PassIter it;
-        it.begin(qt, p.w, p.band);
+        it.begin(qt + p.q_off / kBM, p.w, p.band);
         bool ok = true;
         int qphase[2] = {0, 0};
         auto issue_s = [&](int t, int jj, int kind_changed) -> bool {
@@ -494,14 +496,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-bool make_map(CUtensorMap *m, const void *base, int B, int L, int H) {
+bool make_map(CUtensorMap *m, const void *base, int B, int L, int H, int64_t stride_L = 0) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHD), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHD) * 2,
                                  static_cast<cuuint64_t>(H) * kHD * 2,
-                                 static_cast<cuuint64_t>(L) * H * kHD * 2};
+                                 static_cast<cuuint64_t>(stride_L > 0 ? stride_L : L) * H * kHD * 2};
   const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBN), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
@@ -525,8 +527,13 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
   CUtensorMap mks, mkr, mv;
   const void *krem = a.krem ? a.krem : a.kstd;
   const void *kstd = a.kstd ? a.kstd : a.krem;
-  if (!make_map(&mks, kstd, a.B, a.L, a.Hkv) || !make_map(&mkr, krem, a.B, a.L, a.Hkv) ||
-      !make_map(&mv, a.v, a.B, a.L, a.Hkv))
+  // keys [0, q_off + L); the cache-resident tensors (K_std, V) may be longer
+  // per batch entry than that (kv_stride keys)
+  const int keys = a.q_off + a.L;
+  const int64_t kvs = a.kv_stride > 0 ? a.kv_stride : keys;
+  if (!make_map(&mks, kstd, a.B, keys, a.Hkv, a.kstd ? kvs : keys) ||
+      !make_map(&mkr, krem, a.B, keys, a.Hkv, a.krem ? keys : kvs) ||
+      !make_map(&mv, a.v, a.B, keys, a.Hkv, kvs))
     return cudaErrorInvalidValue;
   KParams p;
   p.q = static_cast<const __nv_bfloat16 *>(a.q);
@@ -541,6 +548,7 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
   p.G = a.G;
   p.w = a.w_eff;
   p.band = a.band;
+  p.q_off = a.q_off;
   p.n_qtiles = (a.L + kBM - 1) / kBM;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * (a.Hq / 2);

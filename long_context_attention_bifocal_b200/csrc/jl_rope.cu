@@ -90,6 +90,47 @@ __global__ void rotate_keys_kernel(const __nv_bfloat16 *__restrict__ k,
   }
 }
 
+// krem[b, k] = R(f(k) - k) kc[b, k] for keys k < L of a cache rotated at
+// original positions: by -u theta_i with u = k - f(k) >= 0, i.e. with the
+// table row u and the sine negated.  One thread per 8 pairs of one key row.
+__global__ void correct_keys_kernel(const __nv_bfloat16 *__restrict__ kc,
+                                    __nv_bfloat16 *__restrict__ krem,
+                                    const float2 *__restrict__ cs, int64_t rows, int L, int cap,
+                                    int Hkv, int D, int G) {
+  const int half = D / 2;
+  const int chunks = half / 8;
+  const int64_t n = rows * chunks;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = idx / chunks;  // (b, l, h) of the output, flattened
+    const int c = static_cast<int>(idx - row * chunks);
+    const int h = static_cast<int>(row % Hkv);
+    const int l = static_cast<int>((row / Hkv) % L);
+    const int64_t b = row / (static_cast<int64_t>(Hkv) * L);
+    const int64_t src = ((b * cap + l) * Hkv + h) * D + 8 * c;
+    const int64_t dst = row * D + 8 * c;
+    float x1[8], x2[8];
+    unpack8(*reinterpret_cast<const uint4 *>(kc + src), x1);
+    unpack8(*reinterpret_cast<const uint4 *>(kc + src + half), x2);
+    const int u = l - l / G;
+    const float2 *t = cs + static_cast<int64_t>(u) * half + 8 * c;
+    float y1[8], y2[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float2 r = __ldg(t + e);
+      y1[e] = x1[e] * r.x + x2[e] * r.y;
+      y2[e] = x2[e] * r.x - x1[e] * r.y;
+    }
+    uint4 o1, o2;
+    o1.x = pack2(y1[0], y1[1]); o1.y = pack2(y1[2], y1[3]);
+    o1.z = pack2(y1[4], y1[5]); o1.w = pack2(y1[6], y1[7]);
+    o2.x = pack2(y2[0], y2[1]); o2.y = pack2(y2[2], y2[3]);
+    o2.z = pack2(y2[4], y2[5]); o2.w = pack2(y2[6], y2[7]);
+    *reinterpret_cast<uint4 *>(krem + dst) = o1;
+    *reinterpret_cast<uint4 *>(krem + dst + half) = o2;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_rope_table(float2 *cs, int positions, int D, double base, cudaStream_t s) {
@@ -117,4 +158,19 @@ cudaError_t launch_rotate_keys(const __nv_bfloat16 *k, __nv_bfloat16 *kstd,
   return cudaGetLastError();
 }
 
+}  // namespace jl
+
+namespace jl {
+cudaError_t launch_correct_keys(const __nv_bfloat16 *kc, __nv_bfloat16 *krem, RopeTable t,
+                                int B, int L, int cap, int Hkv, int D, int G, cudaStream_t s) {
+  const int64_t rows = static_cast<int64_t>(B) * L * Hkv;
+  const int64_t n = rows * (D / 16);
+  const int threads = 256;
+  const int64_t want = (n + threads - 1) / threads;
+  const int64_t lim = static_cast<int64_t>(sm_count()) * 16;
+  const int blocks = static_cast<int>(want < lim ? want : lim);
+  if (blocks < 1) return cudaSuccess;
+  correct_keys_kernel<<<blocks, threads, 0, s>>>(kc, krem, t.cs, rows, L, cap, Hkv, D, G);
+  return cudaGetLastError();
+}
 }  // namespace jl

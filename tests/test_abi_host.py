@@ -197,3 +197,29 @@ def test_decode_batched_workspace_size(lib):
     n = lib.jl_bifocal_decode_batched_workspace_size(4, 32, 8, 128)
     assert n >= (148 + 8) * 32 * 132 * 4
     assert lib.jl_bifocal_decode_batched_workspace_size(4, 32, 8, 64) == 0
+
+
+def _prefill_chunk(lib, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, q_offset=256, cap=1024, out=FAKE, lse=FAKE, B=1, Lq=300,
+             Hq=4, Hkv=2, D=128, w_local=64, w_pretrained=128, base=1e6, flags=0, ws=None,
+             ws_bytes=0)
+    a.update(kw)
+    return lib.jl_bifocal_prefill_chunk(a["q"], a["kc"], a["vc"], a["q_offset"], a["cap"],
+                                        a["out"], a["lse"], a["B"], a["Lq"], a["Hq"], a["Hkv"],
+                                        a["D"], a["w_local"], a["w_pretrained"], a["base"],
+                                        a["flags"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q_offset=100), UNSUPPORTED),       # not a multiple of 128
+    (dict(q_offset=-128), UNSUPPORTED),
+    (dict(cap=500), INVALID),                # q_offset + Lq > cap
+    (dict(D=64), UNSUPPORTED),
+    (dict(Lq=0), INVALID),
+    (dict(ws=FAKE, ws_bytes=10), INVALID),
+    (dict(ws=FAKE + 16, ws_bytes=1 << 30), INVALID),
+    (dict(flags=1 << 31), INVALID),
+])
+def test_prefill_chunk_rejects(lib, kw, code):
+    assert _prefill_chunk(lib, **kw) == code
+    assert lib.jl_last_error()
