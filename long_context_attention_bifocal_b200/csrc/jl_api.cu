@@ -615,8 +615,12 @@ jl_status jl_bifocal_decode_batched(const void *q_new, const void *k_cache_roped
 
   // Plan: one wave of CTAs over all keys; each sequence's remote range
   // [0, far_end) and local range [far_end, pos] are cut into chunks of at most
-  // `chunk` keys (a multiple of 16), so at most kDecodeBatchCtas + 2B chunks.
-  long long chunk = (total + kDecodeBatchCtas - 1) / kDecodeBatchCtas;
+  // `chunk` keys (a multiple of 16).  Each range adds at most one partial
+  // chunk, so aiming at kDecodeBatchCtas - 2B chunks keeps the plan within one
+  // wave (up to 66 sequences) and always within kDecodeBatchCtas + 2B.
+  const long long target =
+      kDecodeBatchCtas - 2LL * B > 16 ? kDecodeBatchCtas - 2LL * B : 16;
+  long long chunk = (total + target - 1) / target;
   chunk = ((chunk + 15) / 16) * 16;
   if (chunk < 16) chunk = 16;
   std::vector<DecodeWork> work;

@@ -105,6 +105,9 @@ struct KParams {
   float scale_log2;  // softmax scale * log2(e)
 };
 
+// kGeneral: band passes or a query offset (the unfused three-call path and
+// chunked prefill); the default prefill runs the instantiation without them.
+template <bool kGeneral>
 __global__ void __launch_bounds__(kThreads, 1)
     bifocal_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_kstd,
                                  const __grid_constant__ CUtensorMap tm_krem,
@@ -116,6 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int band = kGeneral ? p.band : kBandNone;
+  const int q_off = kGeneral ? p.q_off : 0;
 
   const int bh = p.B * p.Hq;
   const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x / bh);
@@ -161,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------ softmax warpgroup --
       const int r = threadIdx.x;  // query row within the tile == TMEM lane
       const int row_i = kBM * qt + r;    // row of the q / out / lse tensors
-      const int qpos = p.q_off + row_i;  // its position
+      const int qpos = q_off + row_i;  // its position
       const bool row_ok = row_i < p.L;
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
       const __nv_bfloat16 *qrow =
@@ -201,13 +206,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       {
         PassIter t0;
-        t0.begin(qt + p.q_off / kBM, p.w, p.band);
+        t0.begin(qt + q_off / kBM, p.w, band);
         rotate_q(t0.kind() == kRem ? pos_rem : pos_std);
       }
 
       float m = -INFINITY, l = 0.f;
       PassIter t;
-      t.begin(qt + p.q_off / kBM, p.w, p.band);
+      t.begin(qt + q_off / kBM, p.w, band);
       int it = 0;
       bool ok = true;
       while (!t.done()) {
@@ -225,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         const int k0 = kBN * t.j;
         const int mk = t.mask();
-        const bool causal = (t.j == qt + p.q_off / kBM);
+        const bool causal = (t.j == qt + q_off / kBM);
         const int kind = t.kind();
         t.next();
         if (kind == kRem && !t.done() && t.kind() == kStd)
@@ -372,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_krem);
         prefetch_tmap(&tm_v);
         PassIter t;
-        t.begin(qt + p.q_off / kBM, p.w, p.band);
+        t.begin(qt + q_off / kBM, p.w, band);
         int kiss = 0, viss = 0;  // loads issued
         while (!t.done()) {
           const int s = kiss % kStages;
@@ -432,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         PassIter t;
-        t.begin(qt + p.q_off / kBM, p.w, p.band);
+        t.begin(qt + q_off / kBM, p.w, band);
         int it = 0, qphase = 0, prev_kind = t.kind();
         while (ok && !t.done()) {
           const int kind = t.kind();
@@ -525,8 +530,11 @@ cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(bifocal_prefill_sm100_kernel,
+    attr_err = cudaFuncSetAttribute(bifocal_prefill_sm100_kernel<false>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(bifocal_prefill_sm100_kernel<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   });
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap mks, mkr, mv;
@@ -557,8 +565,10 @@ cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s) {
   p.n_qtiles = (a.L + kBM - 1) / kBM;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * a.Hq;
-  bifocal_prefill_sm100_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(
-      mks, mkr, mv, p);
+  if (a.band != 0 || a.q_off != 0)
+    bifocal_prefill_sm100_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mks, mkr, mv, p);
+  else
+    bifocal_prefill_sm100_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mks, mkr, mv, p);
   return cudaGetLastError();
 }
 

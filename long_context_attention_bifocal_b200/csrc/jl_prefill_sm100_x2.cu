@@ -134,6 +134,9 @@ __device__ __forceinline__ void rotate_q_row(uint8_t *dst, int r, const __nv_bfl
   }
 }
 
+// kGeneral: band passes or a query offset (the unfused three-call path and
+// chunked prefill); the default prefill runs the instantiation without them.
+template <bool kGeneral>
 __global__ void __launch_bounds__(kThreads, 1)
     bifocal_prefill_sm100_x2_kernel(const __grid_constant__ CUtensorMap tm_kstd,
                                     const __grid_constant__ CUtensorMap tm_krem,
@@ -145,6 +148,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int band = kGeneral ? p.band : kBandNone;
+  const int q_off = kGeneral ? p.q_off : 0;
 
   const int pairs = p.Hq / 2;
   const int bp = p.B * pairs;
@@ -192,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r = threadIdx.x & 127;   // query row == TMEM lane
       const int hq = hq0 + t;
       const int row_i = kBM * qt + r;    // row of the q / out / lse tensors
-      const int qpos = p.q_off + row_i;  // its position
+      const int qpos = q_off + row_i;  // its position
       const bool row_ok = row_i < p.L;
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
       const uint32_t s_col = lane_base + tm_s(t);
@@ -204,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int pos_rem = row_ok ? qpos / p.G : 0;
 
       PassIter it;
-      it.begin(qt + p.q_off / kBM, p.w, p.band);
+      it.begin(qt + q_off / kBM, p.w, band);
       // first Q variant = the class of the first pass
       rotate_q_row(qdst, r, qrow, row_ok, p.cs, it.kind() == kRem ? pos_rem : pos_std);
       fence_proxy_async_smem();
@@ -231,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bar(kBarQReady + t));
         }
 
-        const bool causal = (kj == qt + p.q_off / kBM);
+        const bool causal = (kj == qt + q_off / kBM);
         const bool plain = !causal && mk == kMaskNone;
         const int k0 = kBN * kj;
         // validity of column e for this row (only asked on masked tiles)
@@ -370,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_krem);
         prefetch_tmap(&tm_v);
         PassIter it;
-        it.begin(qt + p.q_off / kBM, p.w, p.band);
+        it.begin(qt + q_off / kBM, p.w, band);
         int kiss = 0, viss = 0;
         while (!it.done()) {
           const int s = kiss % kStages;
@@ -417,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // PV_t(j), which has read them.  While head t's softmax runs on S_t(j),
         // the tensor core works on head 1-t.
         PassIter it;
-        it.begin(qt + p.q_off / kBM, p.w, p.band);
+        it.begin(qt + q_off / kBM, p.w, band);
         bool ok = true;
         int qphase[2] = {0, 0};
         auto issue_s = [&](int t, int jj, int kind_changed) -> bool {
@@ -520,8 +525,11 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(bifocal_prefill_sm100_x2_kernel,
+    attr_err = cudaFuncSetAttribute(bifocal_prefill_sm100_x2_kernel<false>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(bifocal_prefill_sm100_x2_kernel<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   });
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap mks, mkr, mv;
@@ -552,8 +560,10 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
   p.n_qtiles = (a.L + kBM - 1) / kBM;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * (a.Hq / 2);
-  bifocal_prefill_sm100_x2_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(
-      mks, mkr, mv, p);
+  if (a.band != 0 || a.q_off != 0)
+    bifocal_prefill_sm100_x2_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mks, mkr, mv, p);
+  else
+    bifocal_prefill_sm100_x2_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mks, mkr, mv, p);
   return cudaGetLastError();
 }
 
