@@ -9,16 +9,22 @@
 // it loads feeds two S = Q K^T and two O += P V products, and the tensor core
 // alternates between the two heads while each head's softmax runs.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax of head 0: thread r = query row r = TMEM lane r of S0/O0
 //   warps 4-7  softmax of head 1: the same on S1/O1
 //   warp 8     TMA producer: K tile (pre-rotated copy of the pass's class) and
 //              V tile into a 2-stage ring
 //   warp 9     TMEM allocation and every tcgen05.mma, from one thread
+//   warps 10-11 idle (they complete the third warpgroup)
+// Registers: launched at 168 a thread; the third warpgroup drops to 72 and the
+// softmax warpgroups rise to 216 (setmaxnreg), so a softmax thread holds its
+// whole S row and reads S from TMEM once per pass.
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.  After the
 // softmax has read S_t into registers it writes P_t (bf16, two per column) into
-// the first 64 columns of S_t, and O_t += P_t V takes P_t straight from TMEM;
-// the next S_t is issued only after that product has completed.
+// the first 64 columns of S_t, and O_t += P_t V takes P_t straight from TMEM.
+// Issue order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): the next S_t follows the
+// product that reads P_t from the same thread, and the tensor core runs one
+// thread's MMAs in order, so no completion wait sits between them.
 //
 // Shared memory holds one Q variant per head: the remote passes of a query
 // tile all come before its local passes, so Q_rem is used first and is then
@@ -26,10 +32,10 @@
 // q_ready barrier).  Q rotation runs in the softmax warps from the cos/sin
 // table; keys arrive already rotated.
 //
-// Exponentials: a fraction of each row's 2^x runs on the FMA pipe as
-// 2^floor(x) * p(x - floor(x)) with a cubic p fitted by least squares
-// (derive_exp2_poly.py, max relative error 1.1e-4), the rest on the MUFU unit,
-// so neither unit alone bounds the softmax.  Masked tiles use MUFU only.
+// Exponentials: MUFU ex2.approx.  A compile-time option (JL_X2_POLY_EVERY)
+// moves a fraction of each unmasked row to 2^floor(x) * p(x - floor(x)) on the
+// FMA pipe (cubic fitted by least squares, derive_exp2_poly.py, max relative
+// error 1.1e-4); it measured slower on a B200 and is off.
 //
 // Every mbarrier wait is bounded; an abandoned wait raises the CTA abort flag
 // and the device status word, all roles drain their in-flight copies and MMAs,
@@ -49,7 +55,7 @@ using namespace sm100;
 using namespace prefill;
 
 constexpr int kStages = 2;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;  // three warpgroups: softmax 0, softmax 1, producer + MMA
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 
@@ -191,6 +197,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool skip = *reinterpret_cast<volatile int *>(smem + kOffSkip) != 0;
 
   if (!skip) {
+    // Registers are launched at 168 a thread; the producer/MMA warpgroup gives
+    // 128 back per thread so that each softmax thread may hold a whole S row
+    // (2 x 128 x 216 + 128 x 72 = 384 x 168).
+    if (warp < 8)
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
+    else
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
     if (warp < 8) {
       // --------------------------------------------- softmax warpgroups --
       const int t = warp >> 2;           // head of this warpgroup
@@ -247,23 +260,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (mk == kMaskLocalOnly) v = v && dd < p.w;
           return v;
         };
-        // pass 1 over S, 64 columns at a time: row max of the raw scores
+        // S once: all 128 columns in registers (masked entries -> -inf)
+        float sv[128];
+        tmem_ld128(s_col, sv);
+        if (!plain) {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) sv[e] = valid(e) ? sv[e] : -INFINITY;
+        }
         float mt;
         {
           float mx[8];
 #pragma unroll
           for (int a = 0; a < 8; ++a) mx[a] = -INFINITY;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            float sv[64];
-            tmem_ld64(s_col + 64 * h, sv);
-            if (!plain) {
-#pragma unroll
-              for (int e = 0; e < 64; ++e) sv[e] = valid(64 * h + e) ? sv[e] : -INFINITY;
-            }
-#pragma unroll
-            for (int e = 0; e < 64; e += 2) mx[(e >> 1) & 7] = fmax3(mx[(e >> 1) & 7], sv[e], sv[e + 1]);
-          }
+          for (int e = 0; e < 128; e += 2) mx[(e >> 1) & 7] = fmax3(mx[(e >> 1) & 7], sv[e], sv[e + 1]);
           mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
                p.scale_log2;  // scale > 0 keeps the order
         }
@@ -275,7 +285,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_new;
           resc = true;
         }
-        // O_t is stable here: its last product was issued before this S and
+        // P = 2^(s * scale * log2(e) - m), written as bf16 into the first 64
+        // columns of S (every S value is already in registers)
+        const float neg_mu = (m == -INFINITY) ? 0.f : -m;
+        float rsum[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) rsum[a] = 0.f;
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2_pack(neg_mu, neg_mu);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int i0 = 32 * c + 2 * e;
+            float p0, p1;
+            if ((e % kPolyEvery) == kPolyEvery - 1 && plain) {
+              const uint64_t x2 = f2_fma(f2_pack(sv[i0], sv[i0 + 1]), sc2, nm2);
+              f2_unpack(exp2_poly2(x2), p0, p1);
+            } else {
+              p0 = ex2_approx(fmaf(sv[i0], p.scale_log2, neg_mu));
+              p1 = ex2_approx(fmaf(sv[i0 + 1], p.scale_log2, neg_mu));
+            }
+            rsum[e & 7] += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          // every S value is in registers, so P may overwrite any S column
+          tmem_st16_nowait(s_col + 16 * c, pk);
+        }
+        tmem_wait_st();
+        // (after P, so that S is no longer live) O_t is stable here: its last product was issued before this S and
         // this S's completion covers it.  The TMEM access is warp-collective.
         if (j > 0 && __any_sync(0xffffffffu, resc && l > 0.f)) {
           const float a = (resc && l > 0.f) ? alpha : 1.f;
@@ -288,50 +327,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(o_col + 32 * c, o);
           }
         }
-        // pass 2 over S, 32 columns at a time: P = 2^(s * scale * log2(e) - m),
-        // written as bf16 into columns of S that are already consumed
-        const float neg_mu = (m == -INFINITY) ? 0.f : -m;
-        float rsum[8];
-#pragma unroll
-        for (int a = 0; a < 8; ++a) rsum[a] = 0.f;
-        // one column pair in kPolyEvery of an unmasked tile takes 2^x on the
-        // FMA pipe: the two softmax warpgroups share each SM sub-partition's
-        // MUFU unit, which would otherwise bound this pass.  Two copies of the
-        // loop, so that neither has a branch inside.
-        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t nm2 = f2_pack(neg_mu, neg_mu);
-        auto exp_pass = [&](auto with_poly) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float sv[32];
-            tmem_ld32(s_col + 32 * c, sv);
-            if (!decltype(with_poly)::value) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) sv[e] = valid(32 * c + e) ? sv[e] : -INFINITY;
-            }
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float p0, p1;
-              if (decltype(with_poly)::value && (e % kPolyEvery) == kPolyEvery - 1) {
-                const uint64_t x2 = f2_fma(f2_pack(sv[2 * e], sv[2 * e + 1]), sc2, nm2);
-                f2_unpack(exp2_poly2(x2), p0, p1);
-              } else {
-                p0 = ex2_approx(fmaf(sv[2 * e], p.scale_log2, neg_mu));
-                p1 = ex2_approx(fmaf(sv[2 * e + 1], p.scale_log2, neg_mu));
-              }
-              rsum[e & 7] += p0 + p1;
-              pk[e] = pack_bf16x2(p0, p1);
-            }
-            // chunk c of P lands on S columns [16c, 16c+16), read by chunks <= c/2
-            tmem_st16_nowait(s_col + 16 * c, pk);
-          }
-        };
-        if (plain)
-          exp_pass(std::true_type{});
-        else
-          exp_pass(std::false_type{});
-        tmem_wait_st();
         const float rs = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) +
                          ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
         l = l * alpha + rs;
@@ -408,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           drain_wait(bar(kBarVFull + d % kStages), (d / kStages) & 1);
       }
       __syncwarp();
-    } else {
+    } else if (warp == kMmaWarp) {
       // ------------------------------------------------------- MMA issuer --
       if (lane == 0) {
         const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
