@@ -288,11 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P = 2^(s * scale * log2(e) - m), written as bf16 into the first 64
         // columns of S (every S value is already in registers)
         const float neg_mu = (m == -INFINITY) ? 0.f : -m;
-        float rsum[8];
-#pragma unroll
-        for (int a = 0; a < 8; ++a) rsum[a] = 0.f;
         const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
         const uint64_t nm2 = f2_pack(neg_mu, neg_mu);
+        uint64_t rsum2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
@@ -300,14 +298,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 16; ++e) {
             const int i0 = 32 * c + 2 * e;
             float p0, p1;
+            const uint64_t x2 = f2_fma(f2_pack(sv[i0], sv[i0 + 1]), sc2, nm2);
             if ((e % kPolyEvery) == kPolyEvery - 1 && plain) {
-              const uint64_t x2 = f2_fma(f2_pack(sv[i0], sv[i0 + 1]), sc2, nm2);
               f2_unpack(exp2_poly2(x2), p0, p1);
             } else {
-              p0 = ex2_approx(fmaf(sv[i0], p.scale_log2, neg_mu));
-              p1 = ex2_approx(fmaf(sv[i0 + 1], p.scale_log2, neg_mu));
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
             }
-            rsum[e & 7] += p0 + p1;
+            rsum2[e & 3] = f2_add(rsum2[e & 3], f2_pack(p0, p1));
             pk[e] = pack_bf16x2(p0, p1);
           }
           // every S value is in registers, so P may overwrite any S column
@@ -327,9 +327,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(o_col + 32 * c, o);
           }
         }
-        const float rs = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) +
-                         ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
+        float rs;
+        {
+          float r0, r1;
+          f2_unpack(f2_add(f2_add(rsum2[0], rsum2[1]), f2_add(rsum2[2], rsum2[3])), r0, r1);
+          rs = r0 + r1;
+        }
         l = l * alpha + rs;
+        // each lane's TMEM stores are complete (waited) and fenced; after the
+        // warp synchronises, one arrival per warp releases them all
         tc_fence_before();
         mbar_arrive(bar(kBarPFull + t));
         ++j;
