@@ -260,14 +260,45 @@ jl_status jl_bifocal_decode_batched(const void *q_new, const void *k_cache_roped
                                     int w_pretrained, double rope_base,
                                     unsigned flags, jl_stream_t stream);
 
+/*
+ * Batched single-token decode over a PAGED cache (the paged form of
+ * jl_bifocal_decode_batched; techwalker §三, bittide §3.3).  Keys and values
+ * live in a shared pool of fixed-size pages; a per-sequence block table lists
+ * the pages of each sequence in key order.
+ *   k_pages, v_pages  DEVICE pools [num_pages, page_size, Hkv, D] bf16; keys
+ *         rotated at their ORIGINAL positions, as in jl_bifocal_decode.
+ *   page_size  keys per page: a positive multiple of 16 (else
+ *         JL_ERR_INVALID_ARG); num_pages * page_size <= 2^31 - 1.
+ *   block_table  DEVICE int32 [B, max_pages_per_seq], 4-byte aligned: key k of
+ *         sequence b is row k % page_size of page
+ *         block_table[b * max_pages_per_seq + k / page_size].  Only the
+ *         entries covering keys 0..pos[b] are read.  An entry outside
+ *         [0, num_pages) is not followed: the kernel reads page 0 instead and
+ *         raises the device status word, so out and lse are invalid and the
+ *         next jl_check_device_status returns JL_ERR_INVALID_ARG.
+ *   pos   HOST array of B positions, 0 <= pos[b] < max_pages_per_seq *
+ *         page_size; the token of sequence b is at pos[b] and already stored.
+ *   q_new, out, lse, workspace, flags: as jl_bifocal_decode_batched (the same
+ *         workspace size; the call is not capturable in a CUDA graph).
+ *   Rows of a page past pos[b] are never used (any contents).  For the same
+ *   keys the result is bit for bit that of jl_bifocal_decode_batched.
+ */
+jl_status jl_bifocal_decode_paged(const void *q_new, const void *k_pages, const void *v_pages,
+                                  int num_pages, int page_size, const int *block_table,
+                                  int max_pages_per_seq, const int *pos, void *out, float *lse,
+                                  void *workspace, size_t workspace_bytes, int B, int Hq,
+                                  int Hkv, int D, int w_local, int w_pretrained,
+                                  double rope_base, unsigned flags, jl_stream_t stream);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 const char *jl_last_error(void);
 
 /*
  * Synchronises `stream`, then reads and clears the current device's status
  * word.  Returns JL_ERR_TIMEOUT if a kernel gave up a bounded wait since the
- * last check (its outputs are then invalid), JL_ERR_CUDA on a CUDA error,
- * JL_OK otherwise.
+ * last check, JL_ERR_INVALID_ARG if a kernel refused an out-of-range index (a
+ * block-table entry of jl_bifocal_decode_paged); the outputs of that call are
+ * then invalid.  JL_ERR_CUDA on a CUDA error, JL_OK otherwise.
  */
 jl_status jl_check_device_status(jl_stream_t stream);
 

@@ -19,7 +19,7 @@ __all__ = [
     "bifocal_prefill_3pass", "prefill_3pass_workspace_size",
     "bifocal_decode_batched", "decode_batched_workspace_size",
     "bifocal_prefill_chunk", "prefill_chunk_workspace_size",
-    "bifocal_decode_noalloc",
+    "bifocal_decode_noalloc", "bifocal_decode_paged",
     "check_device_status", "finalize", "library_path", "load",
 ]
 
@@ -85,6 +85,9 @@ def load():
     L.jl_bifocal_decode_batched.restype = i
     L.jl_bifocal_decode_batched.argtypes = [p, p, p, p, i, p, p, p, sz, i, i, i, i, i, i, d,
                                             u, p]
+    L.jl_bifocal_decode_paged.restype = i
+    L.jl_bifocal_decode_paged.argtypes = [p, p, p, i, i, p, i, p, p, p, p, sz, i, i, i, i, i, i,
+                                          d, u, p]
     L.jl_bifocal_decode_noalloc.restype = i
     L.jl_bifocal_decode_noalloc.argtypes = [p, p, p, i, i, p, p, i, i, i, i, i, i, d, u, p]
     L.jl_last_error.restype = ctypes.c_char_p
@@ -296,6 +299,44 @@ def bifocal_decode_batched(q_new, k_cache, v_cache, pos, *, w_local, w_pretraine
             _ptr(q_new), _ptr(k_cache), _ptr(v_cache), pos_arr, cap, _ptr(out), _ptr(lse),
             _ptr(workspace), workspace.numel(), B, Hq, Hkv, D, int(w_local), int(w_pretrained),
             float(rope_base), int(flags), _stream(stream)))
+    return out, lse
+
+
+def bifocal_decode_paged(q_new, k_pages, v_pages, block_table, pos, *, w_local, w_pretrained,
+                         rope_base, out=None, lse=None, workspace=None, flags=0, stream=None):
+    """Single-token decode of B sequences over a paged cache.  k_pages, v_pages
+    [num_pages, page_size, Hkv, D] bf16 (keys rotated at their original
+    positions); block_table [B, max_pages_per_seq] int32 on the device (page of
+    keys page_size*i .. page_size*(i+1)-1 of sequence b); pos a sequence of B
+    ints.  Returns (out, lse)."""
+    B, Hq, D = q_new.shape
+    num_pages, page_size, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    _need(q_new, "q_new", torch.bfloat16)
+    _need(k_pages, "k_pages", torch.bfloat16, (num_pages, page_size, Hkv, D))
+    _need(v_pages, "v_pages", torch.bfloat16, (num_pages, page_size, Hkv, D))
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError(f"block_table must be [B={B}, max_pages_per_seq]")
+    _need(block_table, "block_table", torch.int32)
+    pos = [int(x) for x in pos]
+    if len(pos) != B:
+        raise ValueError(f"pos must hold {B} positions, got {len(pos)}")
+    pos_arr = (ctypes.c_int * B)(*pos)
+    if out is None:
+        out = torch.empty_like(q_new)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q_new.device)
+    _need(out, "out", torch.bfloat16, (B, Hq, D))
+    _need(lse, "lse", torch.float32, (B, Hq))
+    if workspace is None:
+        workspace = torch.empty(max(decode_batched_workspace_size(B, Hq, Hkv, D), 16),
+                                dtype=torch.uint8, device=q_new.device)
+    _need(workspace, "workspace", torch.uint8)
+    with torch.cuda.device(q_new.device):
+        _check(load().jl_bifocal_decode_paged(
+            _ptr(q_new), _ptr(k_pages), _ptr(v_pages), num_pages, page_size, _ptr(block_table),
+            block_table.shape[1], pos_arr, _ptr(out), _ptr(lse), _ptr(workspace),
+            workspace.numel(), B, Hq, Hkv, D, int(w_local), int(w_pretrained), float(rope_base),
+            int(flags), _stream(stream)))
     return out, lse
 
 

@@ -576,43 +576,27 @@ size_t jl_bifocal_decode_batched_workspace_size(int B, int Hq, int Hkv, int D) {
          n_max * Hq * kDecodePartialFloats * sizeof(float);
 }
 
-jl_status jl_bifocal_decode_batched(const void *q_new, const void *k_cache_roped,
-                                    const void *v_cache, const int *pos, int cache_capacity,
-                                    void *out, float *lse, void *workspace,
-                                    size_t workspace_bytes, int B, int Hq, int Hkv, int D,
-                                    int w_local, int w_pretrained, double rope_base,
-                                    unsigned flags, jl_stream_t stream) {
-  g_last_error.clear();
-  jl_status st = check_common(B, 1, Hq, Hkv, D, w_local, w_pretrained, rope_base);
-  if (st != JL_OK) return st;
-  if (!q_new || !k_cache_roped || !v_cache || !out || !lse || !workspace || !pos)
-    return fail(JL_ERR_INVALID_ARG, "null pointer");
-  if (!aligned16(q_new) || !aligned16(k_cache_roped) || !aligned16(v_cache) ||
-      !aligned16(out) || !aligned16(lse))
-    return fail(JL_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(JL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL)) != 0)
-    return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
-  if (D != 128) return fail(JL_ERR_UNSUPPORTED, "decode supports head dim 128 (got %d)", D);
-  if (!decode_mma_supported(Hq, Hkv, D))
-    return fail(JL_ERR_UNSUPPORTED,
-                "batched decode needs the tensor-core kernel (Hkv <= 8, Hq / Hkv <= 8)");
-  if (cache_capacity < 1) return fail(JL_ERR_INVALID_ARG, "cache_capacity must be >= 1");
+namespace {
+
+// Paged cache of jl_bifocal_decode_paged (null block_table: contiguous caches).
+struct PagedCache {
+  const int *block_table = nullptr;
+  int page_size = 0, max_pages = 0, num_pages = 0;
+};
+
+// Batched decode over host positions `pos` (already validated): plans one wave
+// of CTAs, copies the plan into the workspace and launches.
+jl_status run_decode_batched(const void *q_new, const void *k_cache, const void *v_cache,
+                             const int *pos, int cache_capacity, const PagedCache &pc,
+                             void *out, float *lse, void *workspace, int B, int Hq, int Hkv,
+                             int D, int w_local, int w_pretrained, double rope_base,
+                             unsigned flags, cudaStream_t s) {
   long long total = 0;
   int max_keys = 0;
   for (int b = 0; b < B; ++b) {
-    if (pos[b] < 0 || pos[b] >= cache_capacity)
-      return fail(JL_ERR_INVALID_ARG, "need 0 <= pos[%d] (%d) < cache_capacity (%d)", b, pos[b],
-                  cache_capacity);
     total += static_cast<long long>(pos[b]) + 1;
     max_keys = pos[b] + 1 > max_keys ? pos[b] + 1 : max_keys;
   }
-  const size_t need = jl_bifocal_decode_batched_workspace_size(B, Hq, Hkv, D);
-  if (workspace_bytes < need)
-    return fail(JL_ERR_INVALID_ARG, "workspace too small: %zu bytes, need %zu", workspace_bytes,
-                need);
-
   // Plan: one wave of CTAs over all keys; each sequence's remote range
   // [0, far_end) and local range [far_end, pos] are cut into chunks of at most
   // `chunk` keys (a multiple of 16).  Each range adds at most one partial
@@ -661,10 +645,9 @@ jl_status jl_bifocal_decode_batched(const void *q_new, const void *k_cache_roped
   std::memcpy(tables.data(), work.data(), work.size() * sizeof(DecodeWork));
   std::memcpy(tables.data() + work_bytes, seqs.data(), B * sizeof(DecodeSeq));
 
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   DecodeArgs a;
   a.q = static_cast<const __nv_bfloat16 *>(q_new);
-  a.kc = static_cast<const __nv_bfloat16 *>(k_cache_roped);
+  a.kc = static_cast<const __nv_bfloat16 *>(k_cache);
   a.vc = static_cast<const __nv_bfloat16 *>(v_cache);
   a.out = static_cast<__nv_bfloat16 *>(out);
   a.lse = lse;
@@ -686,7 +669,11 @@ jl_status jl_bifocal_decode_batched(const void *q_new, const void *k_cache_roped
   a.n_far_chunks = 0;
   a.n_chunks = a.n_work;
   a.scale = static_cast<float>(1.0 / std::sqrt(D));
-  st = rope_table(D, rope_base, max_keys < 64 ? 64 : max_keys, s, &a.table);
+  a.block_table = pc.block_table;
+  a.page_size = pc.page_size;
+  a.max_pages = pc.max_pages;
+  a.num_pages = pc.num_pages;
+  jl_status st = rope_table(D, rope_base, max_keys < 64 ? 64 : max_keys, s, &a.table);
   if (st != JL_OK) return st;
   unsigned *status = nullptr;
   st = status_word(&status);
@@ -696,6 +683,94 @@ jl_status jl_bifocal_decode_batched(const void *q_new, const void *k_cache_roped
   if (e != cudaSuccess) return cuda_fail(e, "decode table copy");
   e = launch_decode_mma(a, status, s);
   return e == cudaSuccess ? JL_OK : cuda_fail(e, "batched decode launch");
+}
+
+// Checks shared by the two batched entry points (everything but the caches).
+jl_status check_batched(const void *q_new, const void *k_cache, const void *v_cache,
+                        const int *pos, void *out, float *lse, void *workspace,
+                        size_t workspace_bytes, int B, int Hq, int Hkv, int D, int w_local,
+                        int w_pretrained, double rope_base, unsigned flags) {
+  jl_status st = check_common(B, 1, Hq, Hkv, D, w_local, w_pretrained, rope_base);
+  if (st != JL_OK) return st;
+  if (!q_new || !k_cache || !v_cache || !out || !lse || !workspace || !pos)
+    return fail(JL_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q_new) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      !aligned16(lse))
+    return fail(JL_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(JL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL)) != 0)
+    return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if (D != 128) return fail(JL_ERR_UNSUPPORTED, "decode supports head dim 128 (got %d)", D);
+  if (!decode_mma_supported(Hq, Hkv, D))
+    return fail(JL_ERR_UNSUPPORTED,
+                "batched decode needs the tensor-core kernel (Hkv <= 8, Hq / Hkv <= 8)");
+  const size_t need = jl_bifocal_decode_batched_workspace_size(B, Hq, Hkv, D);
+  if (workspace_bytes < need)
+    return fail(JL_ERR_INVALID_ARG, "workspace too small: %zu bytes, need %zu", workspace_bytes,
+                need);
+  return JL_OK;
+}
+
+}  // namespace
+
+jl_status jl_bifocal_decode_batched(const void *q_new, const void *k_cache_roped,
+                                    const void *v_cache, const int *pos, int cache_capacity,
+                                    void *out, float *lse, void *workspace,
+                                    size_t workspace_bytes, int B, int Hq, int Hkv, int D,
+                                    int w_local, int w_pretrained, double rope_base,
+                                    unsigned flags, jl_stream_t stream) {
+  g_last_error.clear();
+  jl_status st = check_batched(q_new, k_cache_roped, v_cache, pos, out, lse, workspace,
+                               workspace_bytes, B, Hq, Hkv, D, w_local, w_pretrained,
+                               rope_base, flags);
+  if (st != JL_OK) return st;
+  if (cache_capacity < 1) return fail(JL_ERR_INVALID_ARG, "cache_capacity must be >= 1");
+  for (int b = 0; b < B; ++b)
+    if (pos[b] < 0 || pos[b] >= cache_capacity)
+      return fail(JL_ERR_INVALID_ARG, "need 0 <= pos[%d] (%d) < cache_capacity (%d)", b, pos[b],
+                  cache_capacity);
+  return run_decode_batched(q_new, k_cache_roped, v_cache, pos, cache_capacity, PagedCache{},
+                            out, lse, workspace, B, Hq, Hkv, D, w_local, w_pretrained, rope_base,
+                            flags, reinterpret_cast<cudaStream_t>(stream));
+}
+
+jl_status jl_bifocal_decode_paged(const void *q_new, const void *k_pages, const void *v_pages,
+                                  int num_pages, int page_size, const int *block_table,
+                                  int max_pages_per_seq, const int *pos, void *out, float *lse,
+                                  void *workspace, size_t workspace_bytes, int B, int Hq,
+                                  int Hkv, int D, int w_local, int w_pretrained,
+                                  double rope_base, unsigned flags, jl_stream_t stream) {
+  g_last_error.clear();
+  jl_status st = check_batched(q_new, k_pages, v_pages, pos, out, lse, workspace,
+                               workspace_bytes, B, Hq, Hkv, D, w_local, w_pretrained,
+                               rope_base, flags);
+  if (st != JL_OK) return st;
+  if (!block_table) return fail(JL_ERR_INVALID_ARG, "null pointer");
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) != 0)
+    return fail(JL_ERR_INVALID_ARG, "block_table must be 4-byte aligned");
+  if (page_size < 16 || page_size % 16 != 0)
+    return fail(JL_ERR_INVALID_ARG, "page_size must be a positive multiple of 16 (got %d)",
+                page_size);
+  if (num_pages < 1 || max_pages_per_seq < 1)
+    return fail(JL_ERR_INVALID_ARG, "need num_pages >= 1 and max_pages_per_seq >= 1");
+  if (static_cast<long long>(num_pages) * page_size > INT_MAX)
+    return fail(JL_ERR_INVALID_ARG, "the pool holds more than 2^31 - 1 rows");
+  const long long span = static_cast<long long>(max_pages_per_seq) * page_size;
+  for (int b = 0; b < B; ++b)
+    if (pos[b] < 0 || pos[b] >= span)
+      return fail(JL_ERR_INVALID_ARG,
+                  "need 0 <= pos[%d] (%d) < max_pages_per_seq * page_size (%lld)", b, pos[b],
+                  span);
+  PagedCache pc;
+  pc.block_table = block_table;
+  pc.page_size = page_size;
+  pc.max_pages = max_pages_per_seq;
+  pc.num_pages = num_pages;
+  const int cap = span > INT_MAX ? INT_MAX : static_cast<int>(span);
+  return run_decode_batched(q_new, k_pages, v_pages, pos, cap, pc, out, lse, workspace, B, Hq,
+                            Hkv, D, w_local, w_pretrained, rope_base, flags,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 jl_status jl_bifocal_decode_noalloc(const void *q_new, const void *k_cache_roped,
@@ -761,7 +836,10 @@ jl_status jl_check_device_status(jl_stream_t stream) {
   if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
   if (word != 0) {
     cudaMemset(d->status, 0, sizeof word);
-    return fail(JL_ERR_TIMEOUT, "a kernel abandoned a bounded wait (status 0x%x)", word);
+    if (word & kStatusTimeout)
+      return fail(JL_ERR_TIMEOUT, "a kernel abandoned a bounded wait (status 0x%x)", word);
+    return fail(JL_ERR_INVALID_ARG, "a kernel refused an out-of-range index (status 0x%x)",
+                word);
   }
   return JL_OK;
 }

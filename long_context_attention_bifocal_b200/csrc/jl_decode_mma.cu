@@ -13,7 +13,13 @@
 // 16-key blocks through a 3-stage ring in shared memory: per block and head, K
 // and V as two 64-column boxes with the 128-byte swizzle (so ldmatrix reads
 // are conflict-free), one box per producer lane.  The tensor maps end at key pos, so slots past pos read
-// as zeros and are never touched.  The factor warp writes, per block, the 16
+// as zeros and are never touched.  Blocks start on multiples of 16 keys (keys
+// of the first block before the chunk's first are masked like those past its
+// end), so that with a paged cache (fixed-size pages of a shared pool, a block
+// table per sequence) no block straddles two pages: there the maps cover the
+// whole pool and the producer translates each block's first key through the
+// block table, and a paged call computes bit for bit what a contiguous one
+// does.  The factor warp writes, per block, the 16
 // rows of correction factors (cos, sin)(u theta_i) the block needs (u = k -
 // f(k) grows by at most one per key): row u0 + r is the complex product of the
 // fp32 table row u0 (one 512-byte read per block) and the step row r < 16
@@ -81,6 +87,10 @@ struct Params {
   unsigned long long g_magic;  // ceil(2^64 / G): floor(k / G) = umulhi(k, g_magic), G >= 2
   int skip_first_arrival;  // test-only: withhold the first block (bounded-wait check)
   const DecodeWork *work;  // batched decode: this CTA's entry (nullptr: one position for all)
+  // paged cache (block_table != nullptr): sequence b's key k lives in row
+  // k % page_size of page block_table[b * max_pages + k / page_size] of the pool
+  const int *block_table;
+  int page_size, max_pages, num_pages;
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1,
@@ -189,7 +199,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     pbase = static_cast<int64_t>(b) * p.Hq * p.n_chunks + c;
     pstride = p.n_chunks;
   }
-  const int nblk = (k_end - k_begin + kBlock - 1) / kBlock;
+  // first key of the first block: blocks start on multiples of 16 keys (a
+  // page holds whole blocks)
+  const bool paged = p.block_table != nullptr;
+  const int kb0 = k_begin & ~(kBlock - 1);
+  const int nblk = (k_end - kb0 + kBlock - 1) / kBlock;
 
   auto bar = [&](int i) { return sb + kOffBar + 8u * static_cast<uint32_t>(i); };
   // barriers: full[kStages] (the producer's arrival with the TMA bytes, plus,
@@ -224,11 +238,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t dst_off =
         (is_v ? kKBytes : 0u) + h * kHeadBytes + ((lane & 1) ? kHalfTile : 0u);
     const uint32_t bytes = static_cast<uint32_t>(p.Hkv) * 2 * kHeadBytes;
+    // paged: the page of the next block is read one block ahead, so that its
+    // latency overlaps the wait for a free stage
+    const int *bt = paged ? p.block_table + static_cast<int64_t>(b) * p.max_pages : nullptr;
+    int page_next = (paged && nblk > 0) ? __ldg(bt + kb0 / p.page_size) : 0;
     int issued = 0;
     // test-only: no block is loaded, so the consumers' first wait expires
     for (int blk = p.skip_first_arrival ? nblk : 0; blk < nblk; ++blk) {
       const int s = blk % kStages;
       const uint32_t ph = (blk / kStages) & 1;
+      const int k0 = kb0 + blk * kBlock;
+      int row = k0, bc = b;
+      if (paged) {
+        int page = page_next;
+        if (blk + 1 < nblk) page_next = __ldg(bt + (k0 + kBlock) / p.page_size);
+        if (page < 0 || page >= p.num_pages) {  // refused: read page 0, flag the call
+          if (lane == 0) atomicOr(p.status, kStatusBounds);
+          page = 0;
+        }
+        row = page * p.page_size + k0 % p.page_size;
+        bc = 0;
+      }
       bool ok = true;
       if (lane == 0) {
         ok = mbar_wait(bar(kStages + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs);
@@ -242,8 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       if (h < p.Hkv)
-        tma_load_4d(sb + s * kStageBytes + dst_off, map, bar(s), x, h,
-                    k_begin + blk * kBlock, b);
+        tma_load_4d(sb + s * kStageBytes + dst_off, map, bar(s), x, h, row, bc);
       ++issued;
     }
     // never leave with a copy in flight into this CTA's shared memory
@@ -265,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float4 step[kBlock];
 #pragma unroll
     for (int r = 0; r < kBlock; ++r) step[r] = cs4[r * (kHalf / 2) + lane];
-    int u0 = k_begin - div_g(k_begin, g_magic);
+    int u0 = kb0 - div_g(kb0, g_magic);
     float4 base = cs4[static_cast<int64_t>(u0) * (kHalf / 2) + lane];
     for (int blk = 0; blk < nblk; ++blk) {
       const int s = blk % kStages;
@@ -279,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float4 cb = base;
       if (blk + 1 < nblk) {
-        const int kn = k_begin + (blk + 1) * kBlock;
+        const int kn = kb0 + (blk + 1) * kBlock;
         u0 = kn - div_g(kn, g_magic);
         base = cs4[static_cast<int64_t>(u0) * (kHalf / 2) + lane];
       }
@@ -368,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = false;
       break;
     }
-    const int k0 = k_begin + blk * kBlock;
+    const int k0 = kb0 + blk * kBlock;
     const uint32_t kt = sb + s * kStageBytes + hk * kHeadBytes;
     const uint32_t vt = kt + kKBytes;
 
@@ -411,13 +440,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int mt = 0; mt < 8; ++mt)
       ldsm_x4_t(vt + tile_off(vrow, 2 * mt + ((lane >> 3) & 1)), vf[mt][0], vf[mt][1], vf[mt][2],
                 vf[mt][3]);
-    if (k0 + kBlock > k_end) {
-      // keys past the chunk's end: their P is 0, and their V (possibly past a
+    // a block reaching past the chunk's end or starting before its first key
+    const bool edge = k0 + kBlock > k_end || k0 < k_begin;
+    auto in_chunk = [&](int k) { return k >= k_begin && k < k_end; };
+    if (edge) {
+      // keys outside the chunk: their P is 0, and their V (possibly past a
       // sequence's last key, so any value) must not reach O as 0 * inf or NaN
-      const uint32_t m0 = (k0 + 2 * cq < k_end ? 0x0000FFFFu : 0u) |
-                          (k0 + 2 * cq + 1 < k_end ? 0xFFFF0000u : 0u);
-      const uint32_t m1 = (k0 + 8 + 2 * cq < k_end ? 0x0000FFFFu : 0u) |
-                          (k0 + 9 + 2 * cq < k_end ? 0xFFFF0000u : 0u);
+      const uint32_t m0 = (in_chunk(k0 + 2 * cq) ? 0x0000FFFFu : 0u) |
+                          (in_chunk(k0 + 2 * cq + 1) ? 0xFFFF0000u : 0u);
+      const uint32_t m1 = (in_chunk(k0 + 8 + 2 * cq) ? 0x0000FFFFu : 0u) |
+                          (in_chunk(k0 + 9 + 2 * cq) ? 0xFFFF0000u : 0u);
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
         vf[mt][0] &= m0;
@@ -440,9 +472,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     float sv[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) sv[e] = sa[e] + sc[e];
-    if (k0 + kBlock > k_end) {
-      if (k0 + g >= k_end) sv[0] = sv[1] = -INFINITY;
-      if (k0 + g + 8 >= k_end) sv[2] = sv[3] = -INFINITY;
+    if (edge) {
+      if (!in_chunk(k0 + g)) sv[0] = sv[1] = -INFINITY;
+      if (!in_chunk(k0 + g + 8)) sv[2] = sv[3] = -INFINITY;
     }
     float alpha[2];
 #pragma unroll
@@ -574,12 +606,20 @@ cudaError_t launch_decode_mma(const DecodeArgs &a, unsigned *status, cudaStream_
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  // the maps end at the last valid key (of the longest sequence when batched)
-  const int keys = a.work != nullptr ? a.max_keys : a.pos + 1;
+  // the maps end at the last valid key (of the longest sequence when
+  // batched); a paged pool is one sequence of num_pages * page_size rows
   CUtensorMap mk, mv;
-  if (!make_cache_map(&mk, a.kc, a.B, a.cap, keys, a.Hkv) ||
-      !make_cache_map(&mv, a.vc, a.B, a.cap, keys, a.Hkv))
-    return cudaErrorInvalidValue;
+  if (a.block_table != nullptr) {
+    const int rows = a.num_pages * a.page_size;
+    if (!make_cache_map(&mk, a.kc, 1, rows, rows, a.Hkv) ||
+        !make_cache_map(&mv, a.vc, 1, rows, rows, a.Hkv))
+      return cudaErrorInvalidValue;
+  } else {
+    const int keys = a.work != nullptr ? a.max_keys : a.pos + 1;
+    if (!make_cache_map(&mk, a.kc, a.B, a.cap, keys, a.Hkv) ||
+        !make_cache_map(&mv, a.vc, a.B, a.cap, keys, a.Hkv))
+      return cudaErrorInvalidValue;
+  }
   Params p;
   p.q = a.q;
   p.cs = a.table.cs;
@@ -598,6 +638,10 @@ cudaError_t launch_decode_mma(const DecodeArgs &a, unsigned *status, cudaStream_
   p.skip_first_arrival = a.debug_skip_arrival ? 1 : 0;
   p.g_magic = a.G >= 2 ? (~0ull / static_cast<unsigned long long>(a.G)) + 1ull : 0ull;
   p.work = a.work;
+  p.block_table = a.block_table;
+  p.page_size = a.page_size;
+  p.max_pages = a.max_pages;
+  p.num_pages = a.num_pages;
   const dim3 grid = a.work != nullptr ? dim3(a.n_work) : dim3(a.n_chunks, a.B);
   bifocal_decode_mma_kernel<<<grid, kThreads, kSmemAlloc, s>>>(mk, mv, p);
   cudaError_t e = cudaGetLastError();

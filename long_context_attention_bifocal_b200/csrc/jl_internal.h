@@ -112,6 +112,10 @@ struct DecodeArgs {
   const DecodeWork *work = nullptr;
   const DecodeSeq *seqs = nullptr;
   int n_work = 0, max_keys = 0;
+  // paged cache (batched decode only): kc / vc are pools of num_pages pages of
+  // page_size rows [page_size, Hkv, D]; block_table [B, max_pages] on the device
+  const int *block_table = nullptr;
+  int page_size = 0, max_pages = 0, num_pages = 0;
 };
 
 

@@ -223,3 +223,40 @@ def _prefill_chunk(lib, **kw):
 def test_prefill_chunk_rejects(lib, kw, code):
     assert _prefill_chunk(lib, **kw) == code
     assert lib.jl_last_error()
+
+
+def _decode_paged(lib, pos=(100, 5), **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, num_pages=64, page_size=16, bt=FAKE, max_pages=8,
+             out=FAKE, lse=FAKE, ws=FAKE, ws_bytes=1 << 30, B=len(pos) if pos else 2, Hq=8,
+             Hkv=2, D=128, w_local=16, w_pretrained=64, base=1e6, flags=0)
+    a.update(kw)
+    arr = (ctypes.c_int * len(pos))(*pos) if pos is not None else None
+    return lib.jl_bifocal_decode_paged(a["q"], a["kc"], a["vc"], a["num_pages"],
+                                       a["page_size"], a["bt"], a["max_pages"], arr, a["out"],
+                                       a["lse"], a["ws"], a["ws_bytes"], a["B"], a["Hq"],
+                                       a["Hkv"], a["D"], a["w_local"], a["w_pretrained"],
+                                       a["base"], a["flags"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(pos=(100, 128)), INVALID),          # pos >= max_pages * page_size
+    (dict(pos=(100, -1)), INVALID),
+    (dict(pos=None, B=2), INVALID),
+    (dict(page_size=8), INVALID),             # not a multiple of 16
+    (dict(page_size=40), INVALID),
+    (dict(page_size=0), INVALID),
+    (dict(num_pages=0), INVALID),
+    (dict(max_pages=0), INVALID),
+    (dict(num_pages=1 << 27, page_size=32), INVALID),   # 2^32 rows
+    (dict(bt=None), INVALID),
+    (dict(bt=FAKE + 2), INVALID),             # block table not 4-byte aligned
+    (dict(kc=FAKE + 8), INVALID),
+    (dict(D=64), UNSUPPORTED),
+    (dict(Hq=18, Hkv=2), UNSUPPORTED),
+    (dict(ws_bytes=64), INVALID),
+    (dict(flags=1 << 31), INVALID),
+])
+def test_decode_paged_rejects(lib, kw, code):
+    pos = kw.pop("pos", (100, 5))
+    assert _decode_paged(lib, pos=pos, **kw) == code
+    assert lib.jl_last_error()
