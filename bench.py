@@ -40,6 +40,7 @@ METRIC = "bifocal prefill TFLOP/s & % bf16 peak; decode KV-read GB/s & % HBM"
 # DRAM bytes (read + write) of one full-size launch of the prefill kernel,
 # from ncu (dram__bytes_read.sum + dram__bytes_write.sum, one pass) on B200.
 # Must be re-measured (or set to None) whenever that kernel changes.
+PAGE_SIZE = 16  # keys per page of the paged-cache decode line
 PREFILL_TRAFFIC_BYTES = 44.39e9 + 1.06e9
 PREFILL_CFG = "qwen3_8b_L131072"
 DECODE_CFG = "qwen3_8b_decode_n131072"
@@ -276,6 +277,26 @@ def run_cuda(args):
                                                            workspace=wsb, **kwd), 20)
     batched_bytes = sum(kv_bytes(1, dc["Hkv"], dc["D"], p_ + 1) for p_ in bpos)
     dec_batched = max_over_ranks(dec_batched, world)
+    # the same batch in a paged cache: 16-key pages of a shared pool, in a
+    # seeded random order, one block table row per sequence
+    need = [(p_ + PAGE_SIZE) // PAGE_SIZE for p_ in bpos]
+    perm = torch.randperm(sum(need), generator=torch.Generator().manual_seed(rank_seed(7, rank)))
+    table = torch.full((len(bpos), max(need)), -1, dtype=torch.int32)
+    kpg = torch.empty((sum(need), PAGE_SIZE, dc["Hkv"], dc["D"]), dtype=torch.bfloat16, device=dev)
+    vpg = torch.empty_like(kpg)
+    first = 0
+    for b_, p_ in enumerate(bpos):
+        pages = perm[first:first + need[b_]]
+        first += need[b_]
+        table[b_, :need[b_]] = pages.to(torch.int32)
+        idx = pages.to(dev)
+        kpg[idx] = kb[b_, :need[b_] * PAGE_SIZE].reshape(need[b_], PAGE_SIZE, dc["Hkv"], dc["D"])
+        vpg[idx] = vb[b_, :need[b_] * PAGE_SIZE].reshape(need[b_], PAGE_SIZE, dc["Hkv"], dc["D"])
+    table = table.to(dev)
+    dec_paged = avg_ms(lambda: jl.bifocal_decode_paged(qb, kpg, vpg, table, bpos, out=outb,
+                                                       lse=lseb, workspace=wsb, **kwd), 20)
+    dec_paged = max_over_ranks(dec_paged, world)
+    del kpg, vpg, table
     del qb, kb, vb, wsb, outb, lseb
     pre_plain = avg_ms(lambda: prefill(jl.NO_BIFOCAL), max(1, min(3, args.steps)))
     pre_bif = avg_ms(lambda: prefill(0), max(1, min(3, args.steps)))
@@ -361,6 +382,14 @@ def run_cuda(args):
             "value": round(batched_bytes * world / (dec_batched / 1e3) / 1e9, 1),
             "unit": "GB/s",
             "frac_hbm": round(batched_bytes / (dec_batched / 1e3) / 1e9 / hbm, 4),
+        },
+        "decode_paged": {
+            "B": len(bpos), "positions": bpos, "page_size": PAGE_SIZE,
+            "pages": "shuffled pool, seeded",
+            "us_per_call": round(dec_paged * 1e3, 2),
+            "value": round(batched_bytes * world / (dec_paged / 1e3) / 1e9, 1),
+            "unit": "GB/s",
+            "frac_hbm": round(batched_bytes / (dec_paged / 1e3) / 1e9 / hbm, 4),
         },
         "prefill_unfused_3pass": {
             "ms_per_call": round(pre_3pass, 3),

@@ -65,8 +65,9 @@ constexpr int kMaxGroup = 8;          // query heads per kv head (MMA columns)
 constexpr int kThreads = (kMaxHeads + 2) * 32;
 constexpr int kProducerWarp = kMaxHeads;
 constexpr int kFactorWarp = kMaxHeads + 1;
-constexpr uint32_t kHalfTile = kBlock * 128;          // one 64-column box: 2 KiB
+constexpr uint32_t kHalfTile = kBlock * 128;          // 64 dims of one head: 2 KiB
 constexpr uint32_t kHeadBytes = 2 * kHalfTile;        // K (or V) of one head: 4 KiB
+constexpr uint32_t kHalfBytes = kMaxHeads * kHalfTile;  // one 64-dim half, all heads
 constexpr uint32_t kKBytes = kMaxHeads * kHeadBytes;  // 32 KiB
 constexpr uint32_t kTabRow = 32 * 8;                  // 32 x (cos, cos | sin, sin) bf16x2
 constexpr uint32_t kTabBytes = kBlock * kTabRow;      // 16 rows: 4 KiB
@@ -145,9 +146,10 @@ __device__ __forceinline__ void rotate_pairs_bf(uint32_t &lo, uint32_t &hi, uint
 }
 
 // byte offset of 16-byte chunk `ch` (0..15 over the 128 dims) of key row `row`
-// in a head's [2 halves][16 keys][128 B] swizzled tile
+// in a stage's K (or V) laid out [2 halves][heads][16 keys][128 B], swizzled,
+// relative to the head's first row of half 0
 __device__ __forceinline__ uint32_t tile_off(int row, int ch) {
-  return static_cast<uint32_t>((ch >> 3) * kHalfTile + row * 128 + (((ch & 7) ^ (row & 7)) << 4));
+  return static_cast<uint32_t>((ch >> 3) * kHalfBytes + row * 128 + (((ch & 7) ^ (row & 7)) << 4));
 }
 
 __device__ __forceinline__ bool warp_wait_u(uint32_t bar, uint32_t parity,
@@ -223,41 +225,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (*abort_s) return;
 
   if (warp == kProducerWarp) {
-    // One box per lane: lane j loads (head j / 4) K or V (j & 2), dims
-    // 0-63 or 64-127 (j & 1).  Issued by 32 lanes at once, the 32 copies of a
-    // block leave in a few cycles; a single issuing thread would take ~80
-    // cycles per copy and bound the kernel.
+    // Four boxes per block, one per lane 0-3: K or V (lane & 2), dims 0-63
+    // or 64-127 (lane & 1), all kv heads and 16 keys in one box (the maps
+    // order the dimensions dims, keys, heads, so a box lands as [heads][16
+    // keys][128 B]).  Each copy costs the TMA unit tens of cycles to issue
+    // whatever its size, so a few large copies keep the producer off the
+    // critical path.
     if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
     }
-    const int h = lane >> 2;
     const bool is_v = (lane & 2) != 0;
     const int x = (lane & 1) * kHalf;
     const CUtensorMap *map = is_v ? &tm_v : &tm_k;
-    const uint32_t dst_off =
-        (is_v ? kKBytes : 0u) + h * kHeadBytes + ((lane & 1) ? kHalfTile : 0u);
+    const uint32_t dst_off = (is_v ? kKBytes : 0u) + ((lane & 1) ? kHalfBytes : 0u);
     const uint32_t bytes = static_cast<uint32_t>(p.Hkv) * 2 * kHeadBytes;
-    // paged: the page of the next block is read one block ahead, so that its
+    // paged: the logical page and offset of the block advance by 16 keys a
+    // block; a page's entry is read one block before it is needed, so that its
     // latency overlaps the wait for a free stage
     const int *bt = paged ? p.block_table + static_cast<int64_t>(b) * p.max_pages : nullptr;
-    int page_next = (paged && nblk > 0) ? __ldg(bt + kb0 / p.page_size) : 0;
+    int lp = paged ? kb0 / p.page_size : 0;
+    int off = paged ? kb0 - lp * p.page_size : 0;
+    int page_next = (paged && nblk > 0) ? __ldg(bt + lp) : 0;
     int issued = 0;
     // test-only: no block is loaded, so the consumers' first wait expires
     for (int blk = p.skip_first_arrival ? nblk : 0; blk < nblk; ++blk) {
       const int s = blk % kStages;
       const uint32_t ph = (blk / kStages) & 1;
-      const int k0 = kb0 + blk * kBlock;
-      int row = k0, bc = b;
+      int row = kb0 + blk * kBlock, bc = b;
       if (paged) {
         int page = page_next;
-        if (blk + 1 < nblk) page_next = __ldg(bt + (k0 + kBlock) / p.page_size);
         if (page < 0 || page >= p.num_pages) {  // refused: read page 0, flag the call
           if (lane == 0) atomicOr(p.status, kStatusBounds);
           page = 0;
         }
-        row = page * p.page_size + k0 % p.page_size;
+        row = page * p.page_size + off;
         bc = 0;
+        off += kBlock;
+        if (off == p.page_size) {
+          off = 0;
+          ++lp;
+          if (blk + 1 < nblk) page_next = __ldg(bt + lp);
+        }
       }
       bool ok = true;
       if (lane == 0) {
@@ -271,8 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         break;
       }
-      if (h < p.Hkv)
-        tma_load_4d(sb + s * kStageBytes + dst_off, map, bar(s), x, h, row, bc);
+      if (lane < 4) tma_load_4d(sb + s * kStageBytes + dst_off, map, bar(s), x, row, 0, bc);
       ++issued;
     }
     // never leave with a copy in flight into this CTA's shared memory
@@ -398,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       break;
     }
     const int k0 = kb0 + blk * kBlock;
-    const uint32_t kt = sb + s * kStageBytes + hk * kHeadBytes;
+    const uint32_t kt = sb + s * kStageBytes + hk * kHalfTile;
     const uint32_t vt = kt + kKBytes;
 
     // K fragments kf[ks]: [0] key g, [1] key g+8 (dims 16ks + 2cq + {0,1}),
@@ -562,16 +570,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// cache [B, cap, Hkv, 128] bf16 seen as a 4-D tensor ending at key `keys - 1`
+// cache [B, cap, Hkv, 128] bf16 seen as a 4-D tensor (dims, keys, heads,
+// batch) ending at key `keys - 1`; a box is 64 dims x 16 keys x all heads
 bool make_cache_map(CUtensorMap *m, const void *base, int B, int cap, int keys, int Hkv) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(Hkv),
-                              static_cast<cuuint64_t>(keys), static_cast<cuuint64_t>(B)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kD) * 2,
-                                 static_cast<cuuint64_t>(Hkv) * kD * 2,
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(keys),
+                              static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(Hkv) * kD * 2,
+                                 static_cast<cuuint64_t>(kD) * 2,
                                  static_cast<cuuint64_t>(cap) * Hkv * kD * 2};
-  const cuuint32_t box[4] = {kHalf, 1, kBlock, 1};
+  const cuuint32_t box[4] = {kHalf, kBlock, static_cast<cuuint32_t>(Hkv), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
