@@ -167,6 +167,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // launched as a programmatic dependent of whatever precedes it on the
+  // stream: its CTAs may be scheduled while that kernel finishes, and read
+  // nothing before it has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // this CTA's keys [k_begin, k_end) of sequence b, and where its partials go:
   // query head h of the chunk at (pbase + h * pstride) * kDecodePartialFloats
   int b, k_begin, k_end, pos, G;
@@ -652,8 +656,19 @@ cudaError_t launch_decode_mma(const DecodeArgs &a, unsigned *status, cudaStream_
   p.max_pages = a.max_pages;
   p.num_pages = a.num_pages;
   const dim3 grid = a.work != nullptr ? dim3(a.n_work) : dim3(a.n_chunks, a.B);
-  bifocal_decode_mma_kernel<<<grid, kThreads, kSmemAlloc, s>>>(mk, mv, p);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemAlloc;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, bifocal_decode_mma_kernel, mk, mv, p);
+  if (e != cudaSuccess) return e;
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_decode_combine(a, s);
 }

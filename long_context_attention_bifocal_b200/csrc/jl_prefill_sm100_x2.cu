@@ -21,7 +21,9 @@
 // whole S row and reads S from TMEM once per pass.
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.  After the
 // softmax has read S_t into registers it writes P_t (bf16, two per column) into
-// the first 64 columns of S_t, and O_t += P_t V takes P_t straight from TMEM.
+// the first 64 columns of S_t, and O_t += P_t V takes P_t straight from TMEM,
+// in two parts, each multiplied as soon as the softmax has written it (so half
+// of PV_t runs while the softmax is still on the later keys).
 // Issue order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): the next S_t follows the
 // product that reads P_t from the same thread, and the tensor core runs one
 // thread's MMAs in order, so no completion wait sits between them.
@@ -32,10 +34,12 @@
 // q_ready barrier).  Q rotation runs in the softmax warps from the cos/sin
 // table; keys arrive already rotated.
 //
-// Exponentials: MUFU ex2.approx.  A compile-time option (JL_X2_POLY_EVERY)
-// moves a fraction of each unmasked row to 2^floor(x) * p(x - floor(x)) on the
-// FMA pipe (cubic fitted by least squares, derive_exp2_poly.py, max relative
-// error 1.1e-4); it measured slower on a B200 and is off.
+// Exponentials: MUFU ex2.approx.  A compile-time option (JL_X2_POLY_PAIRS)
+// moves some column pairs of each unmasked row to 2^floor(x) * p(x - floor(x))
+// on the FMA pipe (cubic fitted by least squares, derive_exp2_poly.py, max
+// relative error 1.1e-4).  Measured on a B200 at L = 131072: 4 pairs of 64
+// gained 4% while P went to the PV product in one piece, and lose 2-3% since
+// P is released in two parts; it is off.
 //
 // Every mbarrier wait is bounded; an abandoned wait raises the CTA abort flag
 // and the device status word, all roles drain their in-flight copies and MMAs,
@@ -72,8 +76,10 @@ enum : int {
   kBarVFull = kBarKEmpty + kStages,
   kBarVEmpty = kBarVFull + kStages,
   kBarSFull = kBarVEmpty + kStages,  // [2] per head, tcgen05.commit
-  kBarPFull = kBarSFull + 2,         // [2] per head, 128 arrivals
-  kBarODone = kBarPFull + 2,         // [2] per head, tcgen05.commit
+  // [2][2] per head and part of P, 128 arrivals each; head t's pair at
+  // kBarPFull + 4t (the two heads' barriers in different 32-byte sectors)
+  kBarPFull = kBarSFull + 2,
+  kBarODone = kBarPFull + 8,         // [2] per head, tcgen05.commit
   kBarDrain = kBarODone + 2,
   kNumBars = kBarDrain + 1
 };
@@ -87,13 +93,28 @@ static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
 
-// one column pair in kPolyEvery takes 2^x on the FMA pipe (unmasked tiles);
-// a value above 16 keeps every exponential on the MUFU unit.  Off by default:
-// measured on a B200 at L = 131072, every 4th pair costs 2% and every 2nd 12%.
-#ifndef JL_X2_POLY_EVERY
-#define JL_X2_POLY_EVERY 1000
+// Of the 64 column pairs of an unmasked row, kPolyPairs (spread evenly) take
+// 2^x on the FMA pipe instead of the MUFU unit; 0 keeps every exponential on
+// the MUFU unit.
+#ifndef JL_X2_POLY_PAIRS
+#define JL_X2_POLY_PAIRS 0
 #endif
-constexpr int kPolyEvery = JL_X2_POLY_EVERY;
+constexpr int kPolyPairs = JL_X2_POLY_PAIRS;
+// P is released to the PV product in two parts: the first kPSplit of the four
+// 16-column stores (32 keys each), then the rest.  Measured on a B200 at
+// L = 131072 (ms per call): P in one piece 135, split after 1 store 131, after
+// 2 stores 135, four parts 138.
+#ifndef JL_X2_P_SPLIT
+#define JL_X2_P_SPLIT 1
+#endif
+constexpr int kPSplit = JL_X2_P_SPLIT;
+static_assert(kPSplit >= 1 && kPSplit <= 3, "P split");
+static_assert(kPolyPairs >= 0 && kPolyPairs <= 64, "pairs of a row");
+// pair q in [0, 64) is one of the kPolyPairs (a compile-time constant for the
+// unrolled loop)
+__host__ __device__ constexpr bool poly_pair(int q) {
+  return (q + 1) * kPolyPairs / 64 > q * kPolyPairs / 64;
+}
 __host__ __device__ constexpr uint32_t tm_s(int t) { return 128u * t; }
 __host__ __device__ constexpr uint32_t tm_o(int t) { return 256u + 128u * t; }
 
@@ -173,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(kBarQReady + t), 128);
       mbar_init(bar(kBarSFull + t), 1);
-      mbar_init(bar(kBarPFull + t), 128);
+      for (int c = 0; c < 2; ++c) mbar_init(bar(kBarPFull + 4 * t + c), 128);
       mbar_init(bar(kBarODone + t), 1);
     }
     for (int s = 0; s < kStages; ++s) {
@@ -291,32 +312,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
         const uint64_t nm2 = f2_pack(neg_mu, neg_mu);
         uint64_t rsum2[4] = {0ull, 0ull, 0ull, 0ull};
+        // The exponent pass, in four stores of 32 keys.  P goes to the PV
+        // product in two parts: the first kPSplit stores are released once
+        // they have landed in TMEM (checked after the next store's
+        // exponentials, so the store latency hides under them), and PV_t(j)
+        // starts on them while the softmax is still on the later keys.  kPoly: unmasked tile, where the FMA-pipe 2^x may take
+        // part.  kStream false: a warp that must first rescale O (the lazy
+        // rule moved m) writes all of P, rescales O, then releases the chunks,
+        // so that no part of PV_t(j) reaches O before the rescale.  Both are
+        // compile-time choices per copy, so the unrolled loop has no branch.
+        auto exp_pass = [&](auto poly_tag, auto stream_tag) {
+          constexpr bool kPoly = decltype(poly_tag)::value;
+          constexpr bool kStream = decltype(stream_tag)::value;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int i0 = 32 * c + 2 * e;
-            float p0, p1;
-            const uint64_t x2 = f2_fma(f2_pack(sv[i0], sv[i0 + 1]), sc2, nm2);
-            if ((e % kPolyEvery) == kPolyEvery - 1 && plain) {
-              f2_unpack(exp2_poly2(x2), p0, p1);
-            } else {
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
+            for (int e = 0; e < 16; ++e) {
+              const int i0 = 32 * c + 2 * e;
+              float p0, p1;
+              const uint64_t x2 = f2_fma(f2_pack(sv[i0], sv[i0 + 1]), sc2, nm2);
+              if constexpr (kPoly) {
+                if (poly_pair(16 * c + e)) {
+                  f2_unpack(exp2_poly2(x2), p0, p1);
+                } else {
+                  float x0, x1;
+                  f2_unpack(x2, x0, x1);
+                  p0 = ex2_approx(x0);
+                  p1 = ex2_approx(x1);
+                }
+              } else {
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              rsum2[e & 3] = f2_add(rsum2[e & 3], f2_pack(p0, p1));
+              pk[e] = pack_bf16x2(p0, p1);
             }
-            rsum2[e & 3] = f2_add(rsum2[e & 3], f2_pack(p0, p1));
-            pk[e] = pack_bf16x2(p0, p1);
+            if constexpr (kStream) {
+              if (c == kPSplit) {  // the first part has landed: release it
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(kBarPFull + 4 * t));
+              }
+            }
+            // every S value is in registers, so P may overwrite any S column
+            tmem_st16_nowait(s_col + 16 * c, pk);
           }
-          // every S value is in registers, so P may overwrite any S column
-          tmem_st16_nowait(s_col + 16 * c, pk);
-        }
-        tmem_wait_st();
-        // (after P, so that S is no longer live) O_t is stable here: its last product was issued before this S and
-        // this S's completion covers it.  The TMEM access is warp-collective.
-        if (j > 0 && __any_sync(0xffffffffu, resc && l > 0.f)) {
+          tmem_wait_st();
+        };
+        // O_t is stable during this pass: its last product was issued before
+        // this S, and this S's completion covers it.  The TMEM access is
+        // warp-collective, so the choice is made per warp.
+        const bool rescale_o = j > 0 && __any_sync(0xffffffffu, resc && l > 0.f);
+        if (!rescale_o) {
+          if (kPolyPairs > 0 && plain)
+            exp_pass(std::true_type{}, std::true_type{});
+          else
+            exp_pass(std::false_type{}, std::true_type{});
+          tc_fence_before();
+          mbar_arrive(bar(kBarPFull + 4 * t + 1));
+        } else {
+          exp_pass(std::false_type{}, std::false_type{});
+          // (after P, so that S is no longer live)
           const float a = (resc && l > 0.f) ? alpha : 1.f;
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
@@ -326,6 +385,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 32; ++e) o[e] *= a;
             tmem_st32(o_col + 32 * c, o);
           }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(kBarPFull + 4 * t));
+          mbar_arrive(bar(kBarPFull + 4 * t + 1));
         }
         float rs;
         {
@@ -334,10 +397,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           rs = r0 + r1;
         }
         l = l * alpha + rs;
-        // each lane's TMEM stores are complete (waited) and fenced; after the
-        // warp synchronises, one arrival per warp releases them all
-        tc_fence_before();
-        mbar_arrive(bar(kBarPFull + t));
         ++j;
       }
       ok = __all_sync(0xffffffffu, ok);
@@ -448,15 +507,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         auto issue_pv = [&](int t, int jj) -> bool {
           const int s = jj % kStages;
-          if (!wait(kBarPFull + t, jj & 1)) return false;
           if (t == 0 && !wait(kBarVFull + s, (jj / kStages) & 1)) return false;
-          tc_fence_after();
           const uint32_t vb = sb + kOffV + s * kTileBytes;
+          // P_t arrives in two parts; each is multiplied as soon as it is
+          // released.  Each part's steps are a loop with compile-time bounds
+          // and no exit, so it unrolls into a branch-free issue sequence (one
+          // loop with the second wait inside it measured 4-8% slower).
+          auto steps = [&](auto k0_tag, auto k1_tag) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // 16 keys per step, P_t from TMEM
-            umma_bf16_ts(tmem + tm_o(t), tmem + tm_s(t) + 8 * kk,
-                         sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idesc_pv,
-                         (jj > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = decltype(k0_tag)::value; kk < decltype(k1_tag)::value; ++kk)
+              umma_bf16_ts(tmem + tm_o(t), tmem + tm_s(t) + 8 * kk,
+                           sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024), idesc_pv,
+                           (jj > 0 || kk > 0) ? 1u : 0u);
+          };
+          if (!wait(kBarPFull + 4 * t, jj & 1)) return false;
+          tc_fence_after();
+          steps(std::integral_constant<int, 0>{}, std::integral_constant<int, 2 * kPSplit>{});
+          if (!wait(kBarPFull + 4 * t + 1, jj & 1)) return false;
+          tc_fence_after();
+          steps(std::integral_constant<int, 2 * kPSplit>{}, std::integral_constant<int, 8>{});
           umma_commit(bar(kBarODone + t));
           if (t == 1) umma_commit(bar(kBarVEmpty + s));
           return true;
