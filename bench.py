@@ -41,7 +41,7 @@ METRIC = "bifocal prefill TFLOP/s & % bf16 peak; decode KV-read GB/s & % HBM"
 # from ncu (dram__bytes_read.sum + dram__bytes_write.sum, one pass) on B200.
 # Must be re-measured (or set to None) whenever that kernel changes.
 PAGE_SIZE = 16  # keys per page of the paged-cache decode line
-PREFILL_TRAFFIC_BYTES = 70.80e9 + 1.06e9
+PREFILL_TRAFFIC_BYTES = 4.99e9 + 1.07e9
 PREFILL_CFG = "qwen3_8b_L131072"
 DECODE_CFG = "qwen3_8b_decode_n131072"
 

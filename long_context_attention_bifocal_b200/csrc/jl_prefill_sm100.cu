@@ -122,12 +122,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int band = kGeneral ? p.band : kBandNone;
   const int q_off = kGeneral ? p.q_off : 0;
 
-  const int bh = p.B * p.Hq;
-  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x / bh);
-  const int rem = static_cast<int>(blockIdx.x % bh);
-  const int hq = rem % p.Hq;
-  const int b = rem / p.Hq;
-  const int hk = hq / (p.Hq / p.Hkv);
+  // CTA order: the query heads of one kv head of one batch entry in turn;
+  // within them the heaviest query tiles first, the heads of a tile next to
+  // each other.  The CTAs that run together then share one kv head and walk
+  // its K/V tiles at nearly the same time, so each tile comes from DRAM about
+  // once per wave of CTAs.
+  const int heads = p.Hq / p.Hkv;
+  const int per_group = p.n_qtiles * heads;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int r_in = static_cast<int>(blockIdx.x) % per_group;
+  const int qt = p.n_qtiles - 1 - r_in / heads;
+  const int hk = grp % p.Hkv;
+  const int hq = hk * heads + r_in % heads;
+  const int b = grp / p.Hkv;
 
   volatile int *abort_s = reinterpret_cast<volatile int *>(smem + kOffAbort);
   volatile unsigned *abort_g = p.status;

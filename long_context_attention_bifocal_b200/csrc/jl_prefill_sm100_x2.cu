@@ -93,6 +93,15 @@ static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
 
+// kv heads whose CTAs are scheduled together (see the CTA order in the
+// kernel).  Measured on a B200 at L = 131072 (DRAM bytes read per launch, ms
+// per call): all 8 kv heads interleaved 80-177 GB, 132 ms; 4 at a time 17 GB,
+// 128.6 ms; 2: 9.2 GB, 128.4 ms; 1: 5.0 GB, 128.1 ms.
+#ifndef JL_X2_KV_PER_GROUP
+#define JL_X2_KV_PER_GROUP 1
+#endif
+constexpr int kKvPerGroup = JL_X2_KV_PER_GROUP;
+
 // Of the 64 column pairs of an unmasked row, kPolyPairs (spread evenly) take
 // 2^x on the FMA pipe instead of the MUFU unit; 0 keeps every exponential on
 // the MUFU unit.
@@ -126,6 +135,7 @@ struct KParams {
   const float2 *cs;
   unsigned *status;
   int B, L, Hq, Hkv, G, w, n_qtiles;
+  int pair_group;  // head pairs whose CTAs are scheduled together (divides Hq / 2)
   int band;   // kBandNone, kBandStd or kBandRem
   int q_off;  // position of query row 0 (a multiple of 128; keys start at 0)
   float scale_log2;
@@ -178,12 +188,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int band = kGeneral ? p.band : kBandNone;
   const int q_off = kGeneral ? p.q_off : 0;
 
+  // CTA order: groups of pair_group head pairs (whole kv heads) of one batch
+  // entry in turn; within a group the heaviest query tiles first, the pairs
+  // of one tile next to each other.  The CTAs that run together then share
+  // one kv head and start their walks over its K/V tiles at nearly the same
+  // time, so each tile comes from DRAM about once per wave of CTAs.
   const int pairs = p.Hq / 2;
-  const int bp = p.B * pairs;
-  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x / bp);
-  const int rem = static_cast<int>(blockIdx.x % bp);
-  const int hq0 = 2 * (rem % pairs);
-  const int b = rem / pairs;
+  const int pg = p.pair_group;
+  const int per_group = p.n_qtiles * pg;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int r_in = static_cast<int>(blockIdx.x) % per_group;
+  const int qt = p.n_qtiles - 1 - r_in / pg;
+  const int hq0 = 2 * ((grp % (pairs / pg)) * pg + r_in % pg);
+  const int b = grp / (pairs / pg);
   const int hk = hq0 / (p.Hq / p.Hkv);
 
   volatile int *abort_s = reinterpret_cast<volatile int *>(smem + kOffAbort);
@@ -628,6 +645,13 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
   p.band = a.band;
   p.q_off = a.q_off;
   p.n_qtiles = (a.L + kBM - 1) / kBM;
+  {
+    // whole kv heads per group: kKvPerGroup of them (all when fewer)
+    const int pairs = a.Hq / 2, per_kv = (a.Hq / a.Hkv) / 2;
+    int pg = per_kv * kKvPerGroup;
+    if (pg > pairs || pairs % pg != 0) pg = pairs;
+    p.pair_group = pg;
+  }
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * (a.Hq / 2);
   if (a.band != 0 || a.q_off != 0)
