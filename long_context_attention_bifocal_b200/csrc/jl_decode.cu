@@ -322,22 +322,26 @@ __global__ void __launch_bounds__(kThreads)
 
 // Merges the chunk partials: M = max_c m_c, weights 2^(m_c - M),
 // O = sum_c w_c o_c / sum_c w_c l_c, lse = (M + log2 sum_c w_c l_c) * ln 2.
-// One CTA of 8 warps per (batch, query head, 32-dim slice): every warp takes
-// every eighth chunk, one dim per lane (128-byte loads), and the warps' sums
-// are added in shared memory.  The kernel is launched as a programmatic
+// One CTA of 8 warps per (batch, query head, 32-dim slice): warp w takes the
+// chunks c = w, w + 8, ..., one dim per lane (128-byte loads).  A warp first
+// issues the loads of all its chunks (up to kCombinePerWarp at a time), so the
+// partials cost one memory latency, not one per chunk; it merges them against
+// its own maximum, and the warps' results are merged once more in shared
+// memory with the same rescaling.  The kernel is launched as a programmatic
 // dependent of the split kernel: it may start while that kernel runs and
 // waits (griddepcontrol.wait) until the partials are complete and visible.
 constexpr int kCombineThreads = 256;
 constexpr int kCombineSlice = 32;
 constexpr int kCombineSlices = kD / kCombineSlice;
+constexpr int kCombineWarps = kCombineThreads / 32;
+constexpr int kCombinePerWarp = 24;  // chunks per warp and round (192 per round)
 __global__ void __launch_bounds__(kCombineThreads)
     bifocal_decode_combine_kernel(const float *__restrict__ ws, __nv_bfloat16 *__restrict__ out,
                                   float *__restrict__ lse, int n_chunks, int Hq,
                                   const DecodeSeq *__restrict__ seqs) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  constexpr int kW = kCombineThreads / 32;
-  __shared__ float part[kW][kCombineSlice];
-  __shared__ float wmax[kW], wsum[kW];
+  __shared__ float part[kCombineWarps][kCombineSlice];
+  __shared__ float wmax[kCombineWarps], wsum[kCombineWarps];
   const int bh = blockIdx.x / kCombineSlices, sl = blockIdx.x % kCombineSlices;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   // chunk c of (batch, head) bh at src + c * stride; one position for every
@@ -353,37 +357,59 @@ __global__ void __launch_bounds__(kCombineThreads)
     src = ws + static_cast<int64_t>(bh) * n_chunks * kDecodePartialFloats;
     stride = kDecodePartialFloats;
   }
-  float mx = -INFINITY;
-  for (int c = t; c < n_chunks; c += kCombineThreads)
-    mx = fmaxf(mx, src[c * stride + kD]);
+  // this warp's running merge: maximum, weighted sum of o (this lane's dim)
+  // and of l
+  float M = -INFINITY, acc = 0.f, lsum = 0.f;
+  for (int base = 0; base < n_chunks; base += kCombineWarps * kCombinePerWarp) {
+    float mc[kCombinePerWarp], lc[kCombinePerWarp], oc[kCombinePerWarp];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  if (lane == 0) wmax[warp] = mx;
-  __syncthreads();
-  float M = wmax[0];
+    for (int i = 0; i < kCombinePerWarp; ++i) {
+      const int c = base + warp + kCombineWarps * i;
+      mc[i] = -INFINITY;
+      lc[i] = 0.f;
+      oc[i] = 0.f;
+      if (c < n_chunks) {
+        const float *pc = src + static_cast<int64_t>(c) * stride;
+        mc[i] = pc[kD];
+        lc[i] = pc[kD + 1];
+        oc[i] = pc[kCombineSlice * sl + lane];
+      }
+    }
+    float mr = M;
 #pragma unroll
-  for (int w = 1; w < kW; ++w) M = fmaxf(M, wmax[w]);
-  float acc = 0.f, lsum = 0.f;
-#pragma unroll 4
-  for (int c = warp; c < n_chunks; c += kW) {
-    const float *pc = src + static_cast<int64_t>(c) * stride;
-    const float mc = pc[kD];
-    const float f = (mc == -INFINITY) ? 0.f : ex2(mc - M);
-    acc = fmaf(f, pc[kCombineSlice * sl + lane], acc);
-    lsum = fmaf(f, pc[kD + 1], lsum);
+    for (int i = 0; i < kCombinePerWarp; ++i) mr = fmaxf(mr, mc[i]);
+    if (mr != -INFINITY) {
+      const float r = (M == -INFINITY) ? 0.f : ex2(M - mr);
+      acc *= r;
+      lsum *= r;
+#pragma unroll
+      for (int i = 0; i < kCombinePerWarp; ++i) {
+        const float f = (mc[i] == -INFINITY) ? 0.f : ex2(mc[i] - mr);
+        acc = fmaf(f, oc[i], acc);
+        lsum = fmaf(f, lc[i], lsum);
+      }
+      M = mr;
+    }
   }
   part[warp][lane] = acc;
-  if (lane == 0) wsum[warp] = lsum;
+  if (lane == 0) {
+    wmax[warp] = M;
+    wsum[warp] = lsum;
+  }
   __syncthreads();
   if (t < kCombineSlice) {
+    float Mx = wmax[0];
+#pragma unroll
+    for (int w = 1; w < kCombineWarps; ++w) Mx = fmaxf(Mx, wmax[w]);
     float o = 0.f, L = 0.f;
 #pragma unroll
-    for (int w = 0; w < kW; ++w) {
-      o += part[w][t];
-      L += wsum[w];
+    for (int w = 0; w < kCombineWarps; ++w) {
+      const float f = (wmax[w] == -INFINITY) ? 0.f : ex2(wmax[w] - Mx);
+      o = fmaf(f, part[w][t], o);
+      L = fmaf(f, wsum[w], L);
     }
     out[static_cast<int64_t>(bh) * kD + kCombineSlice * sl + t] = __float2bfloat16_rn(o / L);
-    if (sl == 0 && t == 0) lse[bh] = (M + __log2f(L)) * 0.69314718055994530942f;
+    if (sl == 0 && t == 0) lse[bh] = (Mx + __log2f(L)) * 0.69314718055994530942f;
   }
 }
 

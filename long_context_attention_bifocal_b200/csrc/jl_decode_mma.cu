@@ -598,17 +598,22 @@ bool decode_mma_supported(int Hq, int Hkv, int D) {
   return D == kD && Hkv <= kMaxHeads && Hq / Hkv <= kMaxGroup;
 }
 
-// Keys per CTA: about one wave of CTAs per batch entry, a multiple of the
-// 16-key block; the remote range [0, far_end) and the local range are
-// chunked separately.
+// Keys per CTA: one wave of CTAs per batch entry, a multiple of the 16-key
+// block; the remote range [0, far_end) and the local range are chunked
+// separately, and the chunk grows until both together fit in the wave (a
+// 149th CTA would run after the first ones finish, doubling the tail).
 void decode_mma_plan(int B, int pos, int far_end, int *chunk, int *n_far, int *n_chunks) {
   const long long keys = static_cast<long long>(pos) + 1;
   long long cch = (keys + kCtaTarget - 1) / kCtaTarget;
   cch = ((cch + kBlock - 1) / kBlock) * kBlock;
   if (cch < kBlock) cch = kBlock;
+  auto count = [&](long long c) {
+    return (far_end + c - 1) / c + (keys - far_end + c - 1) / c;
+  };
+  while (count(cch) > kCtaTarget) cch += kBlock;
   *chunk = static_cast<int>(cch);
   *n_far = static_cast<int>((far_end + cch - 1) / cch);
-  *n_chunks = *n_far + static_cast<int>((keys - far_end + cch - 1) / cch);
+  *n_chunks = static_cast<int>(count(cch));
 }
 
 cudaError_t launch_decode_mma(const DecodeArgs &a, unsigned *status, cudaStream_t s) {
