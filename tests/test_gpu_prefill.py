@@ -60,6 +60,9 @@ SMALL = [
     (1, 129, 2, 1, 64, 128, 0.5),      # G=3, window of exactly one tile
     (1, 2125, 4, 1, 1024, 256, 0.5),   # GQA 4, G=3
     (1, 1536, 2, 1, 512, 300, 1.0),    # sharper attention (scores 4x larger)
+    (2, 700, 8, 2, 256, 100, 0.5),     # B=2, two kv heads of two head pairs (CTA order)
+    (1, 600, 6, 2, 200, 64, 0.5),      # GQA 3: odd group, the one-tile kernel
+    (2, 400, 3, 3, 128, 50, 0.5),      # multi-head (group 1), B=2
 ]
 
 
