@@ -507,8 +507,11 @@ def cpu_baseline(q_h, k_h, v_h, qd_h, kc_h, vc_h, kwp, kwd, pos, budget_s=20.0, 
                        W.to_oracle_array(vc_h[:, :pos + 1]), pos, **kwd)
     ddt = time.perf_counter() - t
     kvb = kv_bytes(kc_h.shape[0], kc_h.shape[2], kc_h.shape[3], pos + 1)
+    full = prefill_flops(B, Hq, D, L)
     return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": orc.num_threads(),
             "kind": "oracle",
+            "gflops_fp64": round(fl / dt / 1e9, 2),
+            "full_prefill_s_extrapolated": round(full / (fl / dt), 1),
             "sample": f"prefill: {per_head} seeded rows per query head ({len(rq)} rows) of the "
                       f"L=131072 workload, {dt:.1f} s; decode: the full n=131072 call, "
                       f"{ddt:.1f} s ({kvb / ddt / 1e9:.3f} GB/s)"}
