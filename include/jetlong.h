@@ -34,10 +34,14 @@
  *     and no kernel traps.
  *   - Library-owned device memory: per device, a cos/sin table of the RoPE
  *     angles (fp64 sincos rounded to fp32, [positions][D/2] pairs) grown on
- *     demand, a 4-byte device status word, and, for jl_bifocal_prefill only, a
- *     grown scratch buffer.  jl_finalize releases them.  The first call that
- *     creates or grows them allocates and synchronises, so make it before any
- *     stream capture.
+ *     demand, a 4-byte device status word, and a grown scratch buffer for the
+ *     prefill calls given no workspace.  A table or scratch buffer that is
+ *     replaced by a larger one stays allocated (launches in flight may read
+ *     it) until jl_finalize, which releases them all.  The first call that
+ *     creates or grows them allocates and synchronises its stream, so make it
+ *     before any stream capture.  Prefill calls that use the library's scratch
+ *     buffer and overlap on the GPU (other streams, other threads) race on it:
+ *     serialise them, or give each its own workspace (jl_bifocal_prefill_ex).
  */
 #ifndef JETLONG_H
 #define JETLONG_H

@@ -38,6 +38,9 @@ struct DeviceState {
   unsigned *status = nullptr;
   void *scratch = nullptr;
   size_t scratch_bytes = 0;
+  // buffers replaced by larger ones: another host thread may hold a pointer
+  // to one between taking it and launching, so they live until jl_finalize
+  std::vector<void *> retired;
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -110,10 +113,8 @@ jl_status rope_table(int D, double base, int min_positions, cudaStream_t s, Rope
     if (d->table && d->table_D == D && d->table_base == base && want < 2 * d->table_positions)
       want = 2 * d->table_positions;
     want = ((want + 4095) / 4096) * 4096;
-    if (d->table) {
-      cudaError_t e = cudaDeviceSynchronize();  // earlier kernels may still read it
-      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-      cudaFree(d->table);
+    if (d->table) {  // kept alive: launches in flight or about to start may read it
+      d->retired.push_back(d->table);
       d->table = nullptr;
       d->table_positions = 0;
     }
@@ -152,10 +153,8 @@ jl_status prefill_scratch(size_t bytes, void **out) {
   if (st != JL_OK) return st;
   std::lock_guard<std::mutex> lock(d->mu);
   if (d->scratch_bytes < bytes) {
-    if (d->scratch) {
-      cudaError_t e = cudaDeviceSynchronize();
-      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-      cudaFree(d->scratch);
+    if (d->scratch) {  // kept alive, as the tables are
+      d->retired.push_back(d->scratch);
       d->scratch = nullptr;
       d->scratch_bytes = 0;
     }
@@ -856,6 +855,8 @@ void jl_finalize(void) {
     if (d.table) cudaFree(d.table);
     if (d.status) cudaFree(d.status);
     if (d.scratch) cudaFree(d.scratch);
+    for (void *r : d.retired) cudaFree(r);
+    d.retired.clear();
     d.table = nullptr;
     d.status = nullptr;
     d.scratch = nullptr;
