@@ -17,6 +17,7 @@ CASES = [
     ([5000, 5000, 5000], 6000, 8, 2, 0, 1000),                     # every key remote, G = 6
     ([17, 777, 2100], 2200, 16, 2, 5, 100),                        # GQA 8, G up to 22
     ([129], 200, 4, 4, 64, 32),                                    # B = 1, GQA 1
+    ([3000, 77, 1500], 3100, 8, 1, 300, 700),                      # one kv head, GQA 8
 ]
 
 
@@ -53,3 +54,26 @@ def test_decode_batched_equal_positions_match_single_call(jl):
     jl.check_device_status()
     assert (a[0].float() - b[0].float()).abs().max().item() < 2e-3
     assert (a[1] - b[1]).abs().max().item() < 1e-4
+
+
+def test_decode_batched_many_sequences_two_waves(jl, oracle_mod):
+    """80 short ragged sequences: the plan has more chunks than one wave of
+    CTAs (two chunks per sequence at least), so the kernel runs in waves."""
+    rng = __import__("numpy").random.Generator(__import__("numpy").random.PCG64(5))
+    positions = [int(x) for x in rng.integers(0, 4000, size=80)]
+    B, Hq, Hkv, D, cap = len(positions), 8, 2, 128, 4000
+    q, kc, vc = W.decode_inputs(B, Hq, Hkv, D, cap, seed=77)
+    for b, pos in enumerate(positions):
+        kc[b:b + 1] = poison_tail(kc[b:b + 1], pos)
+        vc[b:b + 1] = poison_tail(vc[b:b + 1], pos)
+    kw = dict(w_local=512, w_pretrained=1024, rope_base=1e6)
+    out, lse = jl.bifocal_decode_batched(q.to(DEV), kc.to(DEV), vc.to(DEV), positions, **kw)
+    jl.check_device_status()
+    orc = oracle_mod.default()
+    for b, pos in enumerate(positions):
+        ref_o, ref_l = orc.bifocal_decode(
+            W.to_oracle_array(q[b:b + 1]), W.to_oracle_array(kc[b:b + 1, :pos + 1]),
+            W.to_oracle_array(vc[b:b + 1, :pos + 1]), pos, **kw)
+        parity.check(parity.to_np(out[b:b + 1]), parity.to_np(lse[b:b + 1]), ref_o, ref_l,
+                     max_abs=parity.BF16_MAX_ABS, mean_abs=parity.BF16_MEAN_ABS,
+                     what=f"sequence {b} at pos {pos}")
