@@ -71,6 +71,16 @@ enum {
    * This is the overhead baseline; with G = 1 the bifocal call takes exactly
    * this path. */
   JL_FLAG_NO_BIFOCAL = 1u << 0,
+  /* jl_bifocal_decode_batched / jl_bifocal_decode_paged: `pos` is a DEVICE
+   * array of B int32 positions (4-byte aligned), read on `stream` when the call
+   * runs.  The plan is then made on the device (no host data, no host
+   * synchronisation), so the call can be captured in a CUDA graph and replayed
+   * with new positions; positions are checked on the device (out of range:
+   * the status word is raised, see jl_check_device_status, and the sequence is
+   * decoded as if at position 0).  The cos/sin table and the tensor maps then
+   * cover the whole cache (cache_capacity, or max_pages_per_seq * page_size),
+   * so make one call before capturing (it may build or grow the table). */
+  JL_FLAG_DEVICE_POS = 1u << 1,
   /* TEST ONLY (jl_bifocal_decode): exercises the kernels' bounded waits.  The
    * decode kernel's TMA producer withholds its first arrival, so the consumer
    * warps' wait on the first K/V block expires after about one second; they
@@ -241,8 +251,9 @@ jl_status jl_bifocal_decode_noalloc(const void *q_new, const void *k_cache_roped
 /*
  * Batched single-token decode, one position per sequence (the batch-size > 1,
  * ragged case of jl_bifocal_decode; techwalker §三, bittide §3.3).
- *   pos   HOST array of B positions, 0 <= pos[b] < cache_capacity; sequence b
- *         decodes its token at pos[b] over cache slots 0..pos[b], with its own
+ *   pos   HOST array of B positions (a DEVICE array with JL_FLAG_DEVICE_POS),
+ *         0 <= pos[b] < cache_capacity; sequence b decodes its token at pos[b]
+ *         over cache slots 0..pos[b], with its own
  *         G = max(1, ceil((pos[b] + 1) / w_pretrained)) and window.
  *   q_new [B, Hq, D], caches [B, cache_capacity, Hkv, D], out [B, Hq, D],
  *   lse [B, Hq]: as jl_bifocal_decode.  Cache slots past pos[b] are never
@@ -250,10 +261,12 @@ jl_status jl_bifocal_decode_noalloc(const void *q_new, const void *k_cache_roped
  *   workspace: at least jl_bifocal_decode_batched_workspace_size() bytes,
  *   256-byte aligned.  The library plans one wave of CTAs over all sequences'
  *   keys on the host and copies the plan (a few KiB, from pageable memory)
- *   into the workspace on `stream` before the kernels; the call is therefore
- *   not capturable in a CUDA graph.
+ *   into the workspace on `stream` before the kernels; such a call is not
+ *   capturable in a CUDA graph.  With JL_FLAG_DEVICE_POS, pos is a device
+ *   array and the same plan is made on the device (capturable, bit for bit
+ *   the same result).
  *   D == 128, Hkv <= 8, Hq / Hkv <= 8 (JL_ERR_UNSUPPORTED otherwise).
- *   flags: JL_FLAG_NO_BIFOCAL.
+ *   flags: JL_FLAG_NO_BIFOCAL, JL_FLAG_DEVICE_POS.
  */
 size_t jl_bifocal_decode_batched_workspace_size(int B, int Hq, int Hkv, int D);
 jl_status jl_bifocal_decode_batched(const void *q_new, const void *k_cache_roped,
@@ -281,9 +294,10 @@ jl_status jl_bifocal_decode_batched(const void *q_new, const void *k_cache_roped
  *         raises the device status word, so out and lse are invalid and the
  *         next jl_check_device_status returns JL_ERR_INVALID_ARG.
  *   pos   HOST array of B positions, 0 <= pos[b] < max_pages_per_seq *
- *         page_size; the token of sequence b is at pos[b] and already stored.
+ *         page_size; the token of sequence b is at pos[b] and already stored
+ *         (a DEVICE array with JL_FLAG_DEVICE_POS).
  *   q_new, out, lse, workspace, flags: as jl_bifocal_decode_batched (the same
- *         workspace size; the call is not capturable in a CUDA graph).
+ *         workspace size; capturable in a CUDA graph with JL_FLAG_DEVICE_POS).
  *   Rows of a page past pos[b] are never used (any contents).  For the same
  *   keys the result is bit for bit that of jl_bifocal_decode_batched.
  */

@@ -14,7 +14,7 @@ import os
 import torch
 
 __all__ = [
-    "NO_BIFOCAL", "DEBUG_SKIP_ARRIVE", "JetLongError", "group_size", "bifocal_prefill",
+    "NO_BIFOCAL", "DEVICE_POS", "DEBUG_SKIP_ARRIVE", "JetLongError", "group_size", "bifocal_prefill",
     "prefill_workspace_size", "decode_workspace_size", "bifocal_decode",
     "bifocal_prefill_3pass", "prefill_3pass_workspace_size",
     "bifocal_decode_batched", "decode_batched_workspace_size",
@@ -24,6 +24,7 @@ __all__ = [
 ]
 
 NO_BIFOCAL = 1 << 0  # JL_FLAG_NO_BIFOCAL
+DEVICE_POS = 1 << 1  # JL_FLAG_DEVICE_POS (set by the bindings when pos is a CUDA tensor)
 DEBUG_SKIP_ARRIVE = 1 << 31  # JL_FLAG_DEBUG_SKIP_ARRIVE (tests of the bounded waits only)
 
 _BF16, _F32 = 0, 1
@@ -127,6 +128,18 @@ def _need(t, name, dtype, shape=None):
         raise ValueError(f"{name} must be contiguous")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _positions(pos, B, flags):
+    """Host positions (a sequence of ints) as a C array, or a CUDA int32 tensor
+    of B positions passed by pointer with JL_FLAG_DEVICE_POS."""
+    if isinstance(pos, torch.Tensor) and pos.is_cuda:
+        _need(pos, "pos", torch.int32, (B,))
+        return ctypes.c_void_p(pos.data_ptr()), int(flags) | DEVICE_POS
+    pos = [int(x) for x in pos]
+    if len(pos) != B:
+        raise ValueError(f"pos must hold {B} positions, got {len(pos)}")
+    return (ctypes.c_int * B)(*pos), int(flags)
 
 
 def group_size(L: int, w_pretrained: int) -> int:
@@ -280,10 +293,7 @@ def bifocal_decode_batched(q_new, k_cache, v_cache, pos, *, w_local, w_pretraine
     _need(q_new, "q_new", torch.bfloat16)
     _need(k_cache, "k_cache", torch.bfloat16, (B, cap, Hkv, D))
     _need(v_cache, "v_cache", torch.bfloat16, (B, cap, Hkv, D))
-    pos = [int(x) for x in pos]
-    if len(pos) != B:
-        raise ValueError(f"pos must hold {B} positions, got {len(pos)}")
-    pos_arr = (ctypes.c_int * B)(*pos)
+    pos_arr, flags = _positions(pos, B, flags)
     if out is None:
         out = torch.empty_like(q_new)
     if lse is None:
@@ -317,10 +327,7 @@ def bifocal_decode_paged(q_new, k_pages, v_pages, block_table, pos, *, w_local, 
     if block_table.dim() != 2 or block_table.shape[0] != B:
         raise ValueError(f"block_table must be [B={B}, max_pages_per_seq]")
     _need(block_table, "block_table", torch.int32)
-    pos = [int(x) for x in pos]
-    if len(pos) != B:
-        raise ValueError(f"pos must hold {B} positions, got {len(pos)}")
-    pos_arr = (ctypes.c_int * B)(*pos)
+    pos_arr, flags = _positions(pos, B, flags)
     if out is None:
         out = torch.empty_like(q_new)
     if lse is None:

@@ -17,7 +17,8 @@ BUILD = os.path.join(ROOT, "_build", "jetlong")
 LIB = os.path.join(PKG, "libjetlong.so")
 
 SOURCES = ["jl_api.cu", "jl_rope.cu", "jl_prefill_sm100.cu", "jl_prefill_sm100_x2.cu",
-           "jl_prefill_f32.cu", "jl_decode.cu", "jl_decode_mma.cu", "jl_merge.cu"]
+           "jl_prefill_f32.cu", "jl_decode.cu", "jl_decode_mma.cu", "jl_merge.cu",
+           "jl_plan.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

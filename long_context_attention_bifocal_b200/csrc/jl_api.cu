@@ -572,7 +572,7 @@ size_t jl_bifocal_decode_batched_workspace_size(int B, int Hq, int Hkv, int D) {
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   const size_t n_max = static_cast<size_t>(kDecodeBatchCtas) + 2 * static_cast<size_t>(B);
   return up(n_max * sizeof(DecodeWork)) + up(static_cast<size_t>(B) * sizeof(DecodeSeq)) +
-         n_max * Hq * kDecodePartialFloats * sizeof(float);
+         up(sizeof(int)) + n_max * Hq * kDecodePartialFloats * sizeof(float);
 }
 
 namespace {
@@ -590,96 +590,119 @@ jl_status run_decode_batched(const void *q_new, const void *k_cache, const void 
                              void *out, float *lse, void *workspace, int B, int Hq, int Hkv,
                              int D, int w_local, int w_pretrained, double rope_base,
                              unsigned flags, cudaStream_t s) {
-  long long total = 0;
-  int max_keys = 0;
-  for (int b = 0; b < B; ++b) {
-    total += static_cast<long long>(pos[b]) + 1;
-    max_keys = pos[b] + 1 > max_keys ? pos[b] + 1 : max_keys;
-  }
-  // Plan: one wave of CTAs over all keys; each sequence's remote range
-  // [0, far_end) and local range [far_end, pos] are cut into chunks of at most
-  // `chunk` keys (a multiple of 16).  Each range adds at most one partial
-  // chunk, so aiming at kDecodeBatchCtas - 2B chunks keeps the plan within one
-  // wave (up to 66 sequences) and always within kDecodeBatchCtas + 2B.
-  const long long target =
-      kDecodeBatchCtas - 2LL * B > 16 ? kDecodeBatchCtas - 2LL * B : 16;
-  long long chunk = (total + target - 1) / target;
-  chunk = ((chunk + 15) / 16) * 16;
-  if (chunk < 16) chunk = 16;
-  std::vector<DecodeWork> work;
-  std::vector<DecodeSeq> seqs(B);
-  for (int b = 0; b < B; ++b) {
-    const int p = pos[b];
-    const long long G = group_size_ll(static_cast<long long>(p) + 1, w_pretrained);
-    const bool plain = (flags & JL_FLAG_NO_BIFOCAL) || G == 1;
-    const long long fe = static_cast<long long>(p) + 1 - w_local;
-    const int far_end = plain ? 0 : static_cast<int>(fe < 0 ? 0 : fe);
-    const unsigned long long magic =
-        G >= 2 ? (~0ull / static_cast<unsigned long long>(G)) + 1ull : 0ull;
-    seqs[b].first = static_cast<int>(work.size());
-    auto cut = [&](int lo, int hi, int far) {
-      for (long long k0 = lo; k0 < hi; k0 += chunk) {
-        DecodeWork w;
-        w.b = b;
-        w.k_begin = static_cast<int>(k0);
-        w.k_end = static_cast<int>(k0 + chunk < hi ? k0 + chunk : hi);
-        w.far = far;
-        w.pos = p;
-        w.G = static_cast<int>(G);
-        w.part = static_cast<int>(work.size()) * Hq;
-        w.pad = 0;
-        w.g_magic = magic;
-        work.push_back(w);
-      }
-    };
-    cut(0, far_end, 1);
-    cut(far_end, p + 1, 0);
-    seqs[b].n = static_cast<int>(work.size()) - seqs[b].first;
-  }
+  const bool pos_on_device = (flags & JL_FLAG_DEVICE_POS) != 0;
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   const size_t n_max = static_cast<size_t>(kDecodeBatchCtas) + 2 * static_cast<size_t>(B);
-  if (work.size() > n_max) return fail(JL_ERR_CUDA, "internal: decode plan too large");
   const size_t work_bytes = up(n_max * sizeof(DecodeWork));
-  std::vector<unsigned char> tables(work_bytes + B * sizeof(DecodeSeq));
-  std::memcpy(tables.data(), work.data(), work.size() * sizeof(DecodeWork));
-  std::memcpy(tables.data() + work_bytes, seqs.data(), B * sizeof(DecodeSeq));
-
+  const size_t seq_bytes = up(B * sizeof(DecodeSeq));
+  char *ws = static_cast<char *>(workspace);
   DecodeArgs a;
   a.q = static_cast<const __nv_bfloat16 *>(q_new);
   a.kc = static_cast<const __nv_bfloat16 *>(k_cache);
   a.vc = static_cast<const __nv_bfloat16 *>(v_cache);
   a.out = static_cast<__nv_bfloat16 *>(out);
   a.lse = lse;
-  char *ws = static_cast<char *>(workspace);
   a.work = reinterpret_cast<const DecodeWork *>(ws);
   a.seqs = reinterpret_cast<const DecodeSeq *>(ws + work_bytes);
-  a.ws = reinterpret_cast<float *>(ws + work_bytes + up(B * sizeof(DecodeSeq)));
-  a.n_work = static_cast<int>(work.size());
-  a.max_keys = max_keys;
+  int *n_work_dev = reinterpret_cast<int *>(ws + work_bytes + seq_bytes);
+  a.ws = reinterpret_cast<float *>(ws + work_bytes + seq_bytes + up(sizeof(int)));
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;
   a.D = D;
-  a.pos = max_keys - 1;
   a.cap = cache_capacity;
   a.G = 1;
   a.far_end = 0;
-  a.chunk = static_cast<int>(chunk);
   a.n_far_chunks = 0;
-  a.n_chunks = a.n_work;
   a.scale = static_cast<float>(1.0 / std::sqrt(D));
   a.block_table = pc.block_table;
   a.page_size = pc.page_size;
   a.max_pages = pc.max_pages;
   a.num_pages = pc.num_pages;
-  jl_status st = rope_table(D, rope_base, max_keys < 64 ? 64 : max_keys, s, &a.table);
-  if (st != JL_OK) return st;
   unsigned *status = nullptr;
-  st = status_word(&status);
+  jl_status st = status_word(&status);
   if (st != JL_OK) return st;
-  // pageable source: the copy is staged before the call returns
-  cudaError_t e = cudaMemcpyAsync(ws, tables.data(), tables.size(), cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return cuda_fail(e, "decode table copy");
+  cudaError_t e = cudaSuccess;
+  std::vector<unsigned char> tables;
+  if (pos_on_device) {
+    // the plan is made on the device: every CTA the plan can hold is launched
+    // and the surplus exit; the maps and the table cover the whole cache
+    a.max_keys = cache_capacity;
+    a.pos = cache_capacity - 1;
+    a.chunk = 16;
+    a.n_work = static_cast<int>(n_max);
+    a.n_chunks = a.n_work;
+    a.n_work_dev = n_work_dev;
+    st = rope_table(D, rope_base, cache_capacity < 64 ? 64 : cache_capacity, s, &a.table);
+    if (st != JL_OK) return st;
+    e = launch_decode_plan(pos, B, cache_capacity, w_local, w_pretrained,
+                           (flags & JL_FLAG_NO_BIFOCAL) != 0, Hq, static_cast<int>(n_max),
+                           reinterpret_cast<DecodeWork *>(ws),
+                           reinterpret_cast<DecodeSeq *>(ws + work_bytes), n_work_dev, status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "decode plan launch");
+  } else {
+    long long total = 0;
+    int max_keys = 0;
+    for (int b = 0; b < B; ++b) {
+      total += static_cast<long long>(pos[b]) + 1;
+      max_keys = pos[b] + 1 > max_keys ? pos[b] + 1 : max_keys;
+    }
+    // Plan: one wave of CTAs over all keys; each sequence's remote range
+    // [0, far_end) and local range [far_end, pos] are cut into chunks of at
+    // most `chunk` keys (a multiple of 16).  Each range adds at most one
+    // partial chunk, so aiming at kDecodeBatchCtas - 2B chunks keeps the plan
+    // within one wave (up to 66 sequences) and always within
+    // kDecodeBatchCtas + 2B.  (jl_plan.cu makes the same plan on the device.)
+    const long long target =
+        kDecodeBatchCtas - 2LL * B > 16 ? kDecodeBatchCtas - 2LL * B : 16;
+    long long chunk = (total + target - 1) / target;
+    chunk = ((chunk + 15) / 16) * 16;
+    if (chunk < 16) chunk = 16;
+    std::vector<DecodeWork> work;
+    std::vector<DecodeSeq> seqs(B);
+    for (int b = 0; b < B; ++b) {
+      const int p = pos[b];
+      const long long G = group_size_ll(static_cast<long long>(p) + 1, w_pretrained);
+      const bool plain = (flags & JL_FLAG_NO_BIFOCAL) || G == 1;
+      const long long fe = static_cast<long long>(p) + 1 - w_local;
+      const int far_end = plain ? 0 : static_cast<int>(fe < 0 ? 0 : fe);
+      const unsigned long long magic =
+          G >= 2 ? (~0ull / static_cast<unsigned long long>(G)) + 1ull : 0ull;
+      seqs[b].first = static_cast<int>(work.size());
+      auto cut = [&](int lo, int hi, int far) {
+        for (long long k0 = lo; k0 < hi; k0 += chunk) {
+          DecodeWork w;
+          w.b = b;
+          w.k_begin = static_cast<int>(k0);
+          w.k_end = static_cast<int>(k0 + chunk < hi ? k0 + chunk : hi);
+          w.far = far;
+          w.pos = p;
+          w.G = static_cast<int>(G);
+          w.part = static_cast<int>(work.size()) * Hq;
+          w.pad = 0;
+          w.g_magic = magic;
+          work.push_back(w);
+        }
+      };
+      cut(0, far_end, 1);
+      cut(far_end, p + 1, 0);
+      seqs[b].n = static_cast<int>(work.size()) - seqs[b].first;
+    }
+    if (work.size() > n_max) return fail(JL_ERR_CUDA, "internal: decode plan too large");
+    tables.resize(work_bytes + B * sizeof(DecodeSeq));
+    std::memcpy(tables.data(), work.data(), work.size() * sizeof(DecodeWork));
+    std::memcpy(tables.data() + work_bytes, seqs.data(), B * sizeof(DecodeSeq));
+    a.max_keys = max_keys;
+    a.pos = max_keys - 1;
+    a.chunk = static_cast<int>(chunk);
+    a.n_work = static_cast<int>(work.size());
+    a.n_chunks = a.n_work;
+    st = rope_table(D, rope_base, max_keys < 64 ? 64 : max_keys, s, &a.table);
+    if (st != JL_OK) return st;
+    // pageable source: the copy is staged before the call returns
+    e = cudaMemcpyAsync(ws, tables.data(), tables.size(), cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "decode table copy");
+  }
   e = launch_decode_mma(a, status, s);
   return e == cudaSuccess ? JL_OK : cuda_fail(e, "batched decode launch");
 }
@@ -698,8 +721,10 @@ jl_status check_batched(const void *q_new, const void *k_cache, const void *v_ca
     return fail(JL_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(JL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL)) != 0)
+  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL | JL_FLAG_DEVICE_POS)) != 0)
     return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if ((flags & JL_FLAG_DEVICE_POS) && (reinterpret_cast<uintptr_t>(pos) & 3u) != 0)
+    return fail(JL_ERR_INVALID_ARG, "device positions must be 4-byte aligned");
   if (D != 128) return fail(JL_ERR_UNSUPPORTED, "decode supports head dim 128 (got %d)", D);
   if (!decode_mma_supported(Hq, Hkv, D))
     return fail(JL_ERR_UNSUPPORTED,
@@ -725,7 +750,7 @@ jl_status jl_bifocal_decode_batched(const void *q_new, const void *k_cache_roped
                                rope_base, flags);
   if (st != JL_OK) return st;
   if (cache_capacity < 1) return fail(JL_ERR_INVALID_ARG, "cache_capacity must be >= 1");
-  for (int b = 0; b < B; ++b)
+  for (int b = 0; b < B && !(flags & JL_FLAG_DEVICE_POS); ++b)
     if (pos[b] < 0 || pos[b] >= cache_capacity)
       return fail(JL_ERR_INVALID_ARG, "need 0 <= pos[%d] (%d) < cache_capacity (%d)", b, pos[b],
                   cache_capacity);
@@ -756,7 +781,7 @@ jl_status jl_bifocal_decode_paged(const void *q_new, const void *k_pages, const 
   if (static_cast<long long>(num_pages) * page_size > INT_MAX)
     return fail(JL_ERR_INVALID_ARG, "the pool holds more than 2^31 - 1 rows");
   const long long span = static_cast<long long>(max_pages_per_seq) * page_size;
-  for (int b = 0; b < B; ++b)
+  for (int b = 0; b < B && !(flags & JL_FLAG_DEVICE_POS); ++b)
     if (pos[b] < 0 || pos[b] >= span)
       return fail(JL_ERR_INVALID_ARG,
                   "need 0 <= pos[%d] (%d) < max_pages_per_seq * page_size (%lld)", b, pos[b],

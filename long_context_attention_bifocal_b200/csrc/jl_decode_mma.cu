@@ -92,6 +92,7 @@ struct Params {
   // k % page_size of page block_table[b * max_pages + k / page_size] of the pool
   const int *block_table;
   int page_size, max_pages, num_pages;
+  const int *n_work_dev;  // plan made on the device: CTAs at or past *n_work_dev exit
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1,
@@ -171,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // stream: its CTAs may be scheduled while that kernel finishes, and read
   // nothing before it has completed
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (p.n_work_dev != nullptr && static_cast<int>(blockIdx.x) >= *p.n_work_dev) return;
   // this CTA's keys [k_begin, k_end) of sequence b, and where its partials go:
   // query head h of the chunk at (pbase + h * pstride) * kDecodePartialFloats
   int b, k_begin, k_end, pos, G;
@@ -660,6 +662,7 @@ cudaError_t launch_decode_mma(const DecodeArgs &a, unsigned *status, cudaStream_
   p.page_size = a.page_size;
   p.max_pages = a.max_pages;
   p.num_pages = a.num_pages;
+  p.n_work_dev = a.n_work_dev;
   const dim3 grid = a.work != nullptr ? dim3(a.n_work) : dim3(a.n_chunks, a.B);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;

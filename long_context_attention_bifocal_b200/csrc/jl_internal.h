@@ -116,7 +116,17 @@ struct DecodeArgs {
   // page_size rows [page_size, Hkv, D]; block_table [B, max_pages] on the device
   const int *block_table = nullptr;
   int page_size = 0, max_pages = 0, num_pages = 0;
+  // plan made on the device: the number of work entries lives here and the
+  // grid has n_work (the most the plan can hold) CTAs; the surplus ones exit
+  const int *n_work_dev = nullptr;
 };
+
+// The batched decode's plan from a device array of positions (one CTA):
+// fills work[0 .. *n_work) and seqs[0 .. B), at most n_max entries.
+cudaError_t launch_decode_plan(const int *pos, int B, int cap, int w_local, int w_pretrained,
+                               bool plain, int Hq, int n_max, DecodeWork *work,
+                               DecodeSeq *seqs, int *n_work, unsigned *status,
+                               cudaStream_t s);
 
 
 // One split partial in the decode workspace: o[128], m (log2 units), l, and
