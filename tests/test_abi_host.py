@@ -260,3 +260,18 @@ def test_decode_paged_rejects(lib, kw, code):
     pos = kw.pop("pos", (100, 5))
     assert _decode_paged(lib, pos=pos, **kw) == code
     assert lib.jl_last_error()
+
+
+def test_decode_batched_device_positions_must_be_aligned(lib):
+    """With JL_FLAG_DEVICE_POS the positions are a device pointer: it must be
+    4-byte aligned (its values are checked on the device, not here)."""
+    B = 2
+    rc = lib.jl_bifocal_decode_batched(FAKE, FAKE, FAKE, ctypes.c_void_p(FAKE + 2), 200, FAKE,
+                                       FAKE, FAKE, 1 << 30, B, 8, 2, 128, 16, 64, 1e6, 1 << 1,
+                                       None)
+    assert rc == INVALID
+    assert lib.jl_last_error()
+    rc = lib.jl_bifocal_decode_paged(FAKE, FAKE, FAKE, 64, 16, FAKE, 8, ctypes.c_void_p(FAKE + 2),
+                                     FAKE, FAKE, FAKE, 1 << 30, B, 8, 2, 128, 16, 64, 1e6, 1 << 1,
+                                     None)
+    assert rc == INVALID
