@@ -277,6 +277,11 @@ def run_cuda(args):
                                                            workspace=wsb, **kwd), 20)
     batched_bytes = sum(kv_bytes(1, dc["Hkv"], dc["D"], p_ + 1) for p_ in bpos)
     dec_batched = max_over_ranks(dec_batched, world)
+    # the same call with the positions on the device (plan made on the GPU)
+    bpos_d = torch.tensor(bpos, dtype=torch.int32, device=dev)
+    dec_batched_dev = avg_ms(lambda: jl.bifocal_decode_batched(qb, kb, vb, bpos_d, out=outb,
+                                                               lse=lseb, workspace=wsb, **kwd), 20)
+    dec_batched_dev = max_over_ranks(dec_batched_dev, world)
     # the same batch in a paged cache: 16-key pages of a shared pool, in a
     # seeded random order, one block table row per sequence
     need = [(p_ + PAGE_SIZE) // PAGE_SIZE for p_ in bpos]
@@ -432,6 +437,7 @@ def run_cuda(args):
             "value": round(batched_bytes * world / (dec_batched / 1e3) / 1e9, 1),
             "unit": "GB/s",
             "frac_hbm": round(batched_bytes / (dec_batched / 1e3) / 1e9 / hbm, 4),
+            "us_per_call_device_positions": round(dec_batched_dev * 1e3, 2),
         },
         "decode_paged": {
             "B": len(bpos), "positions": bpos, "page_size": PAGE_SIZE,
