@@ -285,9 +285,11 @@ def decode_batched_workspace_size(B, Hq, Hkv, D) -> int:
 
 def bifocal_decode_batched(q_new, k_cache, v_cache, pos, *, w_local, w_pretrained, rope_base,
                            out=None, lse=None, workspace=None, flags=0, stream=None):
-    """Single-token decode of B sequences, sequence b at position pos[b] (a
-    sequence of B ints).  q_new [B,Hq,D] pre-RoPE bf16; caches [B,cap,Hkv,D]
-    bf16 with keys rotated at their original positions.  Returns (out, lse)."""
+    """Single-token decode of B sequences, sequence b at position pos[b]: a
+    sequence of B ints, or a CUDA int32 tensor of B positions (the plan is then
+    made on the GPU and the call can be captured in a CUDA graph).  q_new
+    [B,Hq,D] pre-RoPE bf16; caches [B,cap,Hkv,D] bf16 with keys rotated at
+    their original positions.  Returns (out, lse)."""
     B, Hq, D = q_new.shape
     cap, Hkv = k_cache.shape[1], k_cache.shape[2]
     _need(q_new, "q_new", torch.bfloat16)
@@ -318,7 +320,8 @@ def bifocal_decode_paged(q_new, k_pages, v_pages, block_table, pos, *, w_local, 
     [num_pages, page_size, Hkv, D] bf16 (keys rotated at their original
     positions); block_table [B, max_pages_per_seq] int32 on the device (page of
     keys page_size*i .. page_size*(i+1)-1 of sequence b); pos a sequence of B
-    ints.  Returns (out, lse)."""
+    ints or a CUDA int32 tensor (as in bifocal_decode_batched).  Returns
+    (out, lse)."""
     B, Hq, D = q_new.shape
     num_pages, page_size, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
     _need(q_new, "q_new", torch.bfloat16)
