@@ -310,6 +310,25 @@ def pin_zero_query(orc):
         assert np.allclose(lse[h], np.log(np.arange(1, L + 1)), atol=1e-12)
 
 
+def pin_one_hot_values(orc):
+    """V[k] = e_k (one-hot rows, D >= L): O[q] is the attention probability
+    vector of row q itself, so it must be non-negative, sum to 1, vanish after
+    key q (causal), and the first row must attend only to itself."""
+    L, D = 12, 16
+    v = np.zeros((L, 1, D))
+    v[np.arange(L), 0, np.arange(L)] = 1.0
+    q, k = rand((L, 2, D), 81, 2.0), rand((L, 1, D), 82, 2.0)
+    for wl, wp in ((0, 4), (3, 4), (5, 100), (100, 2)):
+        out, _ = run_rows(orc, q, k, v, w_local=wl, w_pretrained=wp, rope_base=1e4)
+        for h in range(2):
+            probs = out[:, h, :L]
+            assert np.all(probs >= 0.0)
+            assert np.allclose(probs.sum(axis=1), 1.0, atol=1e-12)
+            assert np.all(np.triu(probs, 1) == 0.0)   # no key after the query
+            assert np.all(out[:, h, L:] == 0.0)
+            assert probs[0, 0] == 1.0
+
+
 def pin_decode_matches_prefill(orc):
     """Decode over a cache of keys rotated at their original positions, with the
     dq/dk corrections (bittide §3.3), equals the per-pair prefill row L-1."""
@@ -337,5 +356,5 @@ ALL_PINS = [
     pin_rope_complex_form, pin_rope_composition, pin_remote_bound,
     pin_bruteforce, pin_g1_is_plain_rope, pin_all_remote,
     pin_inclusion_exclusion, pin_one_pair_closed_form, pin_zero_query,
-    pin_decode_matches_prefill,
+    pin_one_hot_values, pin_decode_matches_prefill,
 ]
