@@ -18,6 +18,7 @@ CASES = [
     ([17, 777, 2100], 2200, 16, 2, 5, 100),                        # GQA 8, G up to 22
     ([129], 200, 4, 4, 64, 32),                                    # B = 1, GQA 1
     ([3000, 77, 1500], 3100, 8, 1, 300, 700),                      # one kv head, GQA 8
+    ([8191, 4000], 8192, 8, 2, 100, 16),                           # G = 512 and 251
 ]
 
 

@@ -63,6 +63,7 @@ SMALL = [
     (2, 700, 8, 2, 256, 100, 0.5),     # B=2, two kv heads of two head pairs (CTA order)
     (1, 600, 6, 2, 200, 64, 0.5),      # GQA 3: odd group, the one-tile kernel
     (2, 400, 3, 3, 128, 50, 0.5),      # multi-head (group 1), B=2
+    (1, 4096, 2, 1, 16, 100, 0.5),     # G = 256: 256 keys share each remapped position
 ]
 
 
