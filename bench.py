@@ -332,17 +332,26 @@ def run_cuda(args):
     # the pages quote the method as a speed ratio over FlashAttention-2 (plain
     # causal attention of the same shape); the installed flash_attn package,
     # when present, gives that baseline on this GPU (context only)
-    fa2_local, fa2_why = -1.0, None
+    fa2_local, fa2_dec_local, fa2_why = -1.0, -1.0, None
     try:
-        from flash_attn import flash_attn_func
+        from flash_attn import flash_attn_func, flash_attn_with_kvcache
         fa2 = lambda: flash_attn_func(q, k, v, causal=True)  # noqa: E731
         fa2()
         torch.cuda.synchronize()
         fa2_local = avg_ms(fa2, 3)
+        # and its decode over the same cache (one new token per sequence)
+        qd4 = qd.view(dc["B"], 1, dc["Hq"], dc["D"])
+        lens = torch.full((dc["B"],), n, dtype=torch.int32, device=dev)
+        fa2d = lambda: flash_attn_with_kvcache(qd4, kc, vc, cache_seqlens=lens,  # noqa: E731
+                                               causal=True)
+        fa2d()
+        torch.cuda.synchronize()
+        fa2_dec_local = avg_ms(fa2d, 50)
     except Exception as exc:  # the package is optional: report why it is missing
         fa2_why = f"unavailable: {type(exc).__name__}: {str(exc)[:80]}"
     fa2_ms = max_over_ranks(fa2_local, world)  # every rank takes part
-    if fa2_ms < 0 or fa2_why is not None:
+    fa2_dec_ms = max_over_ranks(fa2_dec_local, world)
+    if fa2_ms < 0 or fa2_dec_ms < 0 or fa2_why is not None:
         fa2_ms = fa2_why or "unavailable on some rank"
     jl.check_device_status()
 
@@ -471,7 +480,10 @@ def run_cuda(args):
             {"flashattention2_causal_ms": round(fa2_ms, 3),
              "fused_bifocal_speedup": round(fa2_ms / pre_bif, 3),
              "unfused_3pass_speedup": round(fa2_ms / pre_3pass, 3),
-             "pages_h100": "fused 1.28-1.39x, unfused 0.89-0.93x FlashAttention-2"}
+             "flashattention2_decode_us": round(fa2_dec_ms * 1e3, 2),
+             "bifocal_decode_speedup": round(fa2_dec_ms / dec_bif, 3),
+             "pages_h100": "prefill: fused 1.28-1.39x, unfused 0.89-0.93x; "
+                           "generation: fused 0.96-1.00x FlashAttention-2"}
             if isinstance(fa2_ms, float) else {"flashattention2": fa2_ms}),
         "prefill_chunk": {
             "q_offset": chunk_off, "Lq": chunk_lq, "cache": "the decode workload's",
