@@ -332,8 +332,10 @@ def pin_one_hot_values(orc):
 def pin_decode_matches_prefill(orc):
     """Decode over a cache of keys rotated at their original positions, with the
     dq/dk corrections (bittide §3.3), equals the per-pair prefill row L-1."""
+    # (33, wp=16): pos + 1 = 33 gives G = 3 where pos alone would give 2
     for (L, D, Hq, Hkv, wp, wl) in ((61, 16, 4, 2, 16, 5), (40, 8, 2, 2, 50, 3),
-                                    (100, 32, 2, 1, 25, 0), (77, 8, 1, 1, 10, 200)):
+                                    (100, 32, 2, 1, 25, 0), (77, 8, 1, 1, 10, 200),
+                                    (33, 8, 2, 1, 16, 4)):
         q = rand((L, Hq, D), 71)
         k, v = rand((L, Hkv, D), 72), rand((L, Hkv, D), 73)
         cache = np.stack([np.stack([orc.rope(k[kk, h], kk, 1e6) for h in range(Hkv)])
@@ -351,10 +353,35 @@ def pin_decode_matches_prefill(orc):
         assert np.allclose(l_dec[0], l_pre, atol=1e-11), (L, wl)
 
 
+
+def pin_batch_independence(orc):
+    """Batch elements are separate problems (the method is defined per
+    sequence): a B = 3 call equals three B = 1 calls on the slices, for the
+    prefill rows and for decode over caches whose capacity exceeds pos + 1.
+    The decode slots past pos hold NaN, so reading any of them shows."""
+    L, Hq, Hkv, D = 37, 4, 2, 8
+    kw = dict(w_local=3, w_pretrained=10, rope_base=1e4)
+    q, k, v = rand((3, L, Hq, D), 91), rand((3, L, Hkv, D), 92), rand((3, L, Hkv, D), 93)
+    out, lse = orc.bifocal_all_rows(q, k, v, **kw)
+    for b in range(3):
+        o1, l1 = orc.bifocal_all_rows(q[b:b + 1], k[b:b + 1], v[b:b + 1], **kw)
+        assert np.array_equal(out[b], o1[0]) and np.array_equal(lse[b], l1[0]), b
+    pos, cap = 29, L + 5
+    kc = np.full((3, cap, Hkv, D), np.nan)
+    vc = np.full((3, cap, Hkv, D), np.nan)
+    kc[:, :pos + 1], vc[:, :pos + 1] = k[:, :pos + 1], v[:, :pos + 1]
+    o_dec, l_dec = orc.bifocal_decode(q[:, pos], kc, vc, pos, **kw)
+    assert np.isfinite(o_dec).all() and np.isfinite(l_dec).all()
+    for b in range(3):
+        o1, l1 = orc.bifocal_decode(q[b:b + 1, pos], k[b:b + 1, :pos + 1],
+                                    v[b:b + 1, :pos + 1], pos, **kw)
+        assert np.array_equal(o_dec[b], o1[0]) and np.array_equal(l_dec[b], l1[0]), b
+
+
 ALL_PINS = [
     pin_group_size_golden, pin_group_size_closed_form, pin_rope_closed_form,
     pin_rope_complex_form, pin_rope_composition, pin_remote_bound,
     pin_bruteforce, pin_g1_is_plain_rope, pin_all_remote,
     pin_inclusion_exclusion, pin_one_pair_closed_form, pin_zero_query,
-    pin_one_hot_values, pin_decode_matches_prefill,
+    pin_one_hot_values, pin_decode_matches_prefill, pin_batch_independence,
 ]

@@ -39,6 +39,22 @@ MUTANTS = {
                                    "if (0) {\n          for (int d = 0; d < D; ++d) kc[kk * D + d] = raw[d];"),
     "decode_dk_from_position": ("const double dk = (double)(jlo_remap(kk, G) - kk);",
                                 "const double dk = (double)(jlo_remap(kk, G));"),
+    "decode_group_from_pos": ("jlo_group_size((long long)pos + 1, w_pretrained);",
+                              "jlo_group_size((long long)pos > 0 ? pos : 1, w_pretrained);"),
+    "prefill_keys_ignore_batch": ("const int64_t base = (((int64_t)b * L + kk) * Hkv + hk) * D;",
+                                  "const int64_t base = ((int64_t)kk * Hkv + hk) * D;"),
+    "decode_cache_stride_from_pos": (
+        "const int64_t base = (((int64_t)b * cache_capacity + kk) * Hkv + hk) * D;",
+        "const int64_t base = (((int64_t)b * (pos + 1) + kk) * Hkv + hk) * D;"),
+    "remote_query_at_original_position": (
+        "jlo_rope(raw, qr, D, (double)jlo_remap(qp, G), rope_base);",
+        "jlo_rope(raw, qr, D, (double)qp, rope_base);"),
+    "values_read_from_keys": ("vd[kk * D + d] = jlo_load(v, base + d, dtype);",
+                              "vd[kk * D + d] = jlo_load(k, base + d, dtype);"),
+    "default_scale_over_D": ("if (scale <= 0.0) scale = 1.0 / sqrt((double)D);\n  const long long G = jlo_group_size(L,",
+                             "if (scale <= 0.0) scale = 1.0 / (double)D;\n  const long long G = jlo_group_size(L,"),
+    "decode_query_not_rotated_to_pos": ("jlo_rope(raw, qs, D, (double)pos, rope_base);",
+                                        "jlo_rope(raw, qs, D, 0.0, rope_base);"),
     "softmax_normaliser": ("for (int d = 0; d < D; ++d) out[d] /= Z;",
                            "for (int d = 0; d < D; ++d) out[d] /= (Z + 1.0);"),
 }
