@@ -37,10 +37,10 @@ sys.path.insert(0, ROOT)
 from long_context_attention_bifocal_b200 import workloads as W  # noqa: E402
 
 METRIC = "bifocal prefill TFLOP/s & % bf16 peak; decode KV-read GB/s & % HBM"
+PAGE_SIZE = 16  # keys per page of the paged-cache decode line
 # DRAM bytes (read + write) of one full-size launch of the prefill kernel,
 # from ncu (dram__bytes_read.sum + dram__bytes_write.sum, one pass) on B200.
 # Must be re-measured (or set to None) whenever that kernel changes.
-PAGE_SIZE = 16  # keys per page of the paged-cache decode line
 PREFILL_TRAFFIC_BYTES = 4.99e9 + 1.07e9
 PREFILL_CFG = "qwen3_8b_L131072"
 DECODE_CFG = "qwen3_8b_decode_n131072"
@@ -99,26 +99,35 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
+            lines = f.readlines()
         os.unlink(self.path)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return parse_clock_samples(lines)
+
+
+def parse_clock_samples(lines):
+    """Summarises nvidia-smi lines in ClockSampler.QUERY order (csv, no header,
+    no units): median and maximum SM clock, and every throttle reason seen
+    active in any sample.  Lines that do not parse are skipped; None if no
+    line does."""
+    sm, mx, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in lines:
+        parts = [x.strip() for x in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            mx.append(float(parts[2]))
+        except ValueError:
+            continue
+        for n, v in zip(names, parts[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return None
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+            "reasons": sorted(reasons), "samples": len(sm)}
 
 
 def dist_setup(n_gpus):
