@@ -1,7 +1,7 @@
-"""bench.py's host-side arithmetic and parsing, on the CPU: the algorithmic
-FLOP and byte counts the roofline divides by, the peak file with its
-fallback, and the summary of the clock samples taken during the timed
-region."""
+"""bench.py's host-side parts, on the CPU: the algorithmic FLOP and byte
+counts the roofline divides by, the peak file with its fallback, the summary
+of the clock samples taken during the timed region, and the reference arm
+(the CPU oracle timed on a row sample) with its JSON line."""
 import json
 import os
 import sys
@@ -56,3 +56,34 @@ def test_clock_samples_summary():
 def test_single_rank_helpers_need_no_process_group():
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.rank_seed(7, 0) != bench.rank_seed(7, 1)
+
+
+def _bench(env_extra, *argv):
+    import subprocess
+    env = dict(os.environ, **env_extra)
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *argv],
+                          capture_output=True, text=True, env=env, timeout=600)
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` times the CPU oracle on a bounded row
+    sample and prints one JSON line with the base contract's keys."""
+    res = _bench({}, "--impl", "reference", "--steps", "1", "--warmup", "3")
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["metric"] == bench.METRIC
+    assert rec["value"] > 0 and rec["unit"] == "TFLOP/s" and rec["higher_is_better"] is True
+    assert (rec["steps"], rec["warmup"], rec["n_gpus"]) == (1, 3, 1)
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] >= 1
+    assert rec["cpu_baseline"]["value"] == rec["value"]
+    assert rec["e2e"] == {"value": rec["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                          "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    res = _bench({"RANK": "1", "WORLD_SIZE": "2"}, "--impl", "reference", "--steps", "1",
+                 "--warmup", "3")
+    assert res.returncode == 0, res.stderr[-2000:]
+    assert not [l for l in res.stdout.splitlines() if l.startswith("{")]
