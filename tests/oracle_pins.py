@@ -100,6 +100,22 @@ def pin_group_size_golden(orc):
         assert got == int(G), f"G({L},{w})={got}, pages say {G}"
 
 
+def pin_remap_golden(orc):
+    """The pages' merging example: at L = 65536 over a 32768-token window
+    adjacent positions share one number, and the numbers fill the pretrained
+    range exactly (every number in [0, 32768) used by two positions)."""
+    path = os.path.join(HERE, "golden", "remap_example.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    assert rows and rows[0][0] == "L", "missing header"
+    L, w = int(rows[0][1]), int(rows[0][2])
+    G = orc.group_size(L, w)
+    for x, fx in rows[1:]:
+        got = orc.remap(int(x), G)
+        assert got == int(fx), f"f({x})={got} at G={G}, pages say {fx}"
+    counts = np.bincount([orc.remap(x, G) for x in range(L)])
+    assert len(counts) == w and (counts == 2).all()
+
+
 def pin_group_size_closed_form(orc):
     for L in (1, 2, 127, 128, 129, 512, 32767, 32768, 32769, 49152, 65536,
               98304, 131072, 131073):
@@ -379,7 +395,7 @@ def pin_batch_independence(orc):
 
 
 ALL_PINS = [
-    pin_group_size_golden, pin_group_size_closed_form, pin_rope_closed_form,
+    pin_group_size_golden, pin_remap_golden, pin_group_size_closed_form, pin_rope_closed_form,
     pin_rope_complex_form, pin_rope_composition, pin_remote_bound,
     pin_bruteforce, pin_g1_is_plain_rope, pin_all_remote,
     pin_inclusion_exclusion, pin_one_pair_closed_form, pin_zero_query,
