@@ -76,7 +76,8 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 long long group_size_ll(long long L, long long w) {
   if (L < 1 || w < 1) return -1;
-  const long long g = (L + w - 1) / w;
+  // ceil(L / w) without forming L + w - 1, which overflows near LLONG_MAX
+  const long long g = L / w + (L % w != 0 ? 1 : 0);
   return g < 1 ? 1 : g;
 }
 

@@ -47,6 +47,12 @@ def test_group_size_host(lib):
     assert lib.jl_group_size(98304, 32768) == 3
     assert lib.jl_group_size(0, 5) == -1
     assert lib.jl_group_size(5, 0) == -1
+    # no overflow at the top of the 64-bit range
+    big = 2**63 - 1
+    assert lib.jl_group_size(big, 2) == big // 2 + 1
+    assert lib.jl_group_size(big, big) == 1
+    assert lib.jl_group_size(big - 1, big) == 1
+    assert lib.jl_group_size(big, 1) == big
 
 
 def _prefill(lib, **kw):
