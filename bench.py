@@ -236,7 +236,7 @@ def run_cuda(args):
     total_ms = max_over_ranks(total_ms, world)
     pre_sum = max_over_ranks(sum(pre_ms), world)
     dec_sum = max_over_ranks(sum(dec_ms), world)
-    launches = 4 * args.steps  # per step: key rotation + prefill, decode split + combine
+    launches = 4 * args.steps  # per step: key rotation + prefill, decode + combine
 
     # ---------------- overhead vs the same kernels without the bifocal rule ----
     def avg_ms(fn, reps):
