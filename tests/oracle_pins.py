@@ -394,10 +394,43 @@ def pin_batch_independence(orc):
         assert np.array_equal(o_dec[b], o1[0]) and np.array_equal(l_dec[b], l1[0]), b
 
 
+
+def _bf16_exact(x):
+    """fp64 values that bf16 holds exactly, and their bf16 bit patterns
+    (truncation of the fp32 bits; exact because the values are built that way)."""
+    bits32 = x.astype(np.float32).view(np.uint32) & np.uint32(0xFFFF0000)
+    return bits32.view(np.float32).astype(np.float64), (bits32 >> 16).astype(np.uint16)
+
+
+def pin_input_dtypes(orc):
+    """The same values passed as bf16 bit patterns, fp32 or fp64 give the same
+    result (every step is fp64; bf16 is the top half of an fp32 word), for the
+    prefill rows and for decode.  Negative values, subnormal-free magnitudes
+    from 2^-8 to 2^8."""
+    L, Hq, Hkv, D = 29, 2, 1, 8
+    rng = np.random.Generator(np.random.PCG64(97))
+    def vals(shape):
+        return rng.choice([-1.0, 1.0], shape) * np.exp2(rng.uniform(-8, 8, shape))
+    (q, qb), (k, kb), (v, vb) = (_bf16_exact(vals(sh)) for sh in
+                                 ((1, L, Hq, D), (1, L, Hkv, D), (1, L, Hkv, D)))
+    kw = dict(w_local=4, w_pretrained=8, rope_base=1e4)
+    o64, l64 = orc.bifocal_all_rows(q, k, v, **kw)
+    for args in ((qb, kb, vb), (q.astype(np.float32), k.astype(np.float32), v.astype(np.float32))):
+        o, l = orc.bifocal_all_rows(*args, **kw)
+        assert np.array_equal(o, o64) and np.array_equal(l, l64), args[0].dtype
+    pos = L - 1
+    d64 = orc.bifocal_decode(q[:, pos], k, v, pos, **kw)
+    for args in ((qb[:, pos], kb, vb),
+                 (q[:, pos].astype(np.float32), k.astype(np.float32), v.astype(np.float32))):
+        d = orc.bifocal_decode(*args, pos, **kw)
+        assert np.array_equal(d[0], d64[0]) and np.array_equal(d[1], d64[1]), args[0].dtype
+
+
 ALL_PINS = [
     pin_group_size_golden, pin_remap_golden, pin_group_size_closed_form, pin_rope_closed_form,
     pin_rope_complex_form, pin_rope_composition, pin_remote_bound,
     pin_bruteforce, pin_g1_is_plain_rope, pin_all_remote,
     pin_inclusion_exclusion, pin_one_pair_closed_form, pin_zero_query,
     pin_one_hot_values, pin_decode_matches_prefill, pin_batch_independence,
+    pin_input_dtypes,
 ]

@@ -55,6 +55,10 @@ MUTANTS = {
                              "if (scale <= 0.0) scale = 1.0 / (double)D;\n  const long long G = jlo_group_size(L,"),
     "decode_query_not_rotated_to_pos": ("jlo_rope(raw, qs, D, (double)pos, rope_base);",
                                         "jlo_rope(raw, qs, D, 0.0, rope_base);"),
+    "bf16_widening": ("uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]) << 16;",
+                      "uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]) << 15;"),
+    "fp32_read_as_bf16": ("if (dtype == JLO_F32) return (double)((const float *)base)[idx];",
+                          "if (dtype == JLO_F32) return (double)((const uint16_t *)base)[idx];"),
     "softmax_normaliser": ("for (int d = 0; d < D; ++d) out[d] /= Z;",
                            "for (int d = 0; d < D; ++d) out[d] /= (Z + 1.0);"),
 }
