@@ -426,11 +426,24 @@ def pin_input_dtypes(orc):
         assert np.array_equal(d[0], d64[0]) and np.array_equal(d[1], d64[1]), args[0].dtype
 
 
+
+def pin_explicit_scale(orc):
+    """Scores are linear in q (RoPE is a rotation), so an explicit softmax
+    scale s equals the default 1/sqrt(D) applied to q * s * sqrt(D)."""
+    L, Hq, Hkv, D, s = 33, 2, 1, 8, 0.05
+    q, k, v = rand((1, L, Hq, D), 98), rand((1, L, Hkv, D), 99), rand((1, L, Hkv, D), 100)
+    kw = dict(w_local=5, w_pretrained=10, rope_base=1e4)
+    o1, l1 = orc.bifocal_all_rows(q, k, v, scale=s, **kw)
+    o2, l2 = orc.bifocal_all_rows(q * (s * math.sqrt(D)), k, v, **kw)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(l1, l2, atol=1e-12)
+    assert not np.allclose(o1, orc.bifocal_all_rows(q, k, v, **kw)[0], atol=1e-3)
+
+
 ALL_PINS = [
     pin_group_size_golden, pin_remap_golden, pin_group_size_closed_form, pin_rope_closed_form,
     pin_rope_complex_form, pin_rope_composition, pin_remote_bound,
     pin_bruteforce, pin_g1_is_plain_rope, pin_all_remote,
     pin_inclusion_exclusion, pin_one_pair_closed_form, pin_zero_query,
     pin_one_hot_values, pin_decode_matches_prefill, pin_batch_independence,
-    pin_input_dtypes,
+    pin_input_dtypes, pin_explicit_scale,
 ]

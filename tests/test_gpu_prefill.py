@@ -87,6 +87,18 @@ def test_bf16_small_all_rows_one_tile_kernel(jl, oracle_mod, case, monkeypatch):
     test_bf16_small_all_rows(jl, oracle_mod, case)
 
 
+def test_bf16_explicit_softmax_scale(jl, oracle_mod):
+    """A softmax scale given by the caller instead of 1/sqrt(D)."""
+    q, k, v = W.prefill_inputs(1, 700, 4, 2, 128, dtype="bf16", value_scale=0.5, seed=12)
+    kw = dict(w_local=150, w_pretrained=200, rope_base=1e6)
+    out, lse = jl.bifocal_prefill(q.to(DEV), k.to(DEV), v.to(DEV), softmax_scale=0.05, **kw)
+    jl.check_device_status()
+    ref_o, ref_l = oracle_mod.default().bifocal_all_rows(
+        W.to_oracle_array(q), W.to_oracle_array(k), W.to_oracle_array(v), scale=0.05, **kw)
+    parity.check(parity.to_np(out), parity.to_np(lse), ref_o, ref_l,
+                 max_abs=parity.BF16_MAX_ABS, mean_abs=parity.BF16_MEAN_ABS, what="scale 0.05")
+
+
 def test_bf16_g1_bitwise_plain(jl):
     """G = 1 takes exactly the non-bifocal path."""
     q, k, v = W.prefill_inputs(1, 777, 4, 2, 128, seed=7)

@@ -59,6 +59,8 @@ MUTANTS = {
                       "uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]) << 15;"),
     "fp32_read_as_bf16": ("if (dtype == JLO_F32) return (double)((const float *)base)[idx];",
                           "if (dtype == JLO_F32) return (double)((const uint16_t *)base)[idx];"),
+    "explicit_scale_ignored": ("if (scale <= 0.0) scale = 1.0 / sqrt((double)D);\n  const long long G = jlo_group_size(L,",
+                               "scale = 1.0 / sqrt((double)D);\n  const long long G = jlo_group_size(L,"),
     "softmax_normaliser": ("for (int d = 0; d < D; ++d) out[d] /= Z;",
                            "for (int d = 0; d < D; ++d) out[d] /= (Z + 1.0);"),
 }
