@@ -164,6 +164,112 @@ def barrier(world):
         torch.cuda.synchronize()
 
 
+PREFILL_SWEEP = ["qwen3_1p7b_L65536", "qwen3_4b_L16384", "qwen3_4b_L32768", "qwen3_4b_L49152",
+                 "qwen3_4b_L98304", "qwen3_4b_L131072"]
+
+
+def interleaved(stream, fa, fb, reps):
+    """Medians (ms) of fa and fb timed alternately with CUDA events on `stream`
+    (clock drift and neighbours hit both alike)."""
+    ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    eb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for i, ((a0, a1), (b0, b1)) in enumerate(zip(ea, eb)):
+        a0.record(stream)
+        fa(i)
+        a1.record(stream)
+        b0.record(stream)
+        fb(i)
+        b1.record(stream)
+    torch.cuda.synchronize()
+    med = lambda es: sorted(x.elapsed_time(y) for x, y in es)[reps // 2]  # noqa: E731
+    return med(ea), med(eb)
+
+
+def prefill_sweep(jl, dev, stream, world, rank, reps, bf16_sust):
+    """Every prefill configuration besides the headline one: the 1.7B shape at
+    64K and the 4B shape's length sweep.  Per configuration: median ms per call
+    (bifocal and JL_FLAG_NO_BIFOCAL timed alternately), effective TFLOP/s, the
+    fraction of the sustained bf16 peak and the overhead of the bifocal rule."""
+    res = {}
+    for name in PREFILL_SWEEP:
+        c = W.PREFILL[name]
+        B, L, Hq, Hkv, D = c["B"], c["L"], c["Hq"], c["Hkv"], c["D"]
+        kw = dict(w_local=c["w_local"], w_pretrained=c["w_pretrained"], rope_base=c["rope_base"])
+        q, k, v = (t.to(dev) for t in W.prefill_inputs(
+            B, L, Hq, Hkv, D, value_scale=c["value_scale"], seed=rank_seed(c["seed"], rank)))
+        out = torch.empty_like(q)
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+        run = lambda flags: jl.bifocal_prefill(q, k, v, out=out, lse=lse,  # noqa: E731
+                                               flags=flags, **kw)
+        run(0)
+        run(jl.NO_BIFOCAL)
+        bif, plain = interleaved(stream, lambda i: run(0), lambda i: run(jl.NO_BIFOCAL), reps)
+        bif = max_over_ranks(bif, world)
+        plain = max_over_ranks(plain, world)
+        fl = prefill_flops(B, Hq, D, L)
+        tf = fl / (bif / 1e3) / 1e12
+        G = -(-L // c["w_pretrained"])
+        res[name] = {"L": L, "Hq": Hq, "Hkv": Hkv, "G": G, "ms_per_call": round(bif, 3),
+                     "tflops": round(tf * world, 2), "frac_bf16_sustained": round(tf / bf16_sust, 4),
+                     "ms_no_bifocal": round(plain, 3),
+                     "overhead_vs_no_bifocal": round(bif / plain - 1.0, 4)}
+        del q, k, v, out, lse
+    jl.check_device_status()
+    return res
+
+
+def decode_sweep(jl, dev, stream, world, rank, hbm, reps):
+    """The decode configuration's cache lengths n = 8192 ... 131072 (pos = n-1).
+    Each call reads a different one of several caches in turn, enough of them
+    that the others' bytes since its last use exceed three times the L2, so every
+    call reads its keys and values from HBM.  Bifocal and JL_FLAG_NO_BIFOCAL
+    calls alternate; medians of `reps` calls each."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    res = {}
+    for name, c in W.DECODE.items():
+        n, B, Hq, Hkv, D = c["n"], c["B"], c["Hq"], c["Hkv"], c["D"]
+        pos = n - 1
+        kw = dict(w_local=c["w_local"], w_pretrained=c["w_pretrained"], rope_base=c["rope_base"])
+        nbytes = kv_bytes(B, Hkv, D, n)
+        copies = max(2, int(math.ceil(3 * l2 / nbytes)) + 1)
+        q, kc0, vc0 = W.decode_inputs(B, Hq, Hkv, D, n, seed=rank_seed(c["seed"], rank))
+        q = q.to(dev)
+        caches = []
+        for i in range(copies):
+            kc, vc = kc0.to(dev), vc0.to(dev)
+            if i:
+                # distinct bytes per copy (a rotation of the key order), same distribution
+                kc, vc = torch.roll(kc, 17 * i, dims=1), torch.roll(vc, 17 * i, dims=1)
+            caches.append((kc, vc))
+        out = torch.empty_like(q)
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+        ws = torch.empty(jl.decode_workspace_size(B, Hq, Hkv, D, pos), dtype=torch.uint8,
+                         device=dev)
+
+        def call(i, flags):
+            kc, vc = caches[i % copies]
+            jl.bifocal_decode(q, kc, vc, pos, out=out, lse=lse, workspace=ws, flags=flags, **kw)
+        for i in range(2 * copies):
+            call(i, 0)
+            call(i, jl.NO_BIFOCAL)
+        # the two calls of a pair read different caches too
+        bif, plain = interleaved(stream, lambda i: call(2 * i, 0),
+                                 lambda i: call(2 * i + 1, jl.NO_BIFOCAL), reps)
+        bif = max_over_ranks(bif, world)
+        plain = max_over_ranks(plain, world)
+        gbs = nbytes / (bif / 1e3) / 1e9
+        res[name] = {"n": n, "G": -(-n // c["w_pretrained"]), "us_per_call": round(bif * 1e3, 2),
+                     "value": round(gbs * world, 1), "unit": "GB/s",
+                     "frac_hbm": round(gbs / hbm, 4), "us_no_bifocal": round(plain * 1e3, 2),
+                     "overhead_vs_no_bifocal": round(bif / plain - 1.0, 4),
+                     "distinct_caches": copies}
+        del caches, q, out, lse, ws
+    jl.check_device_status()
+    return res
+
+
 def run_cuda(args):
     import long_context_attention_bifocal_b200 as jl
 
@@ -249,24 +355,8 @@ def run_cuda(args):
         torch.cuda.synchronize()
         return sorted(a.elapsed_time(b) for a, b in es)[reps // 2]
 
-    def interleaved_ms(fa, fb, reps):
-        """Medians of fa and fb timed alternately (clock drift hits both)."""
-        ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(reps)]
-        eb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(reps)]
-        for (a0, a1), (b0, b1) in zip(ea, eb):
-            a0.record(stream)
-            fa()
-            a1.record(stream)
-            b0.record(stream)
-            fb()
-            b1.record(stream)
-        torch.cuda.synchronize()
-        med = lambda es: sorted(x.elapsed_time(y) for x, y in es)[reps // 2]  # noqa: E731
-        return med(ea), med(eb)
-
-    dec_bif, dec_plain = interleaved_ms(lambda: decode(0), lambda: decode(jl.NO_BIFOCAL), 100)
+    dec_bif, dec_plain = interleaved(stream, lambda i: decode(0),
+                                     lambda i: decode(jl.NO_BIFOCAL), 100)
 
     # a ragged batch: 8 sequences of one shape at different positions (G 1-4)
     bpos = [16383, 32767, 49151, 65535, 81919, 98303, 114687, 131071]
@@ -364,6 +454,11 @@ def run_cuda(args):
         fa2_ms = fa2_why or "unavailable on some rank"
     jl.check_device_status()
 
+    # ---------------- the other configurations ----------------
+    hbm, bf16_burst, bf16_sust, src = peaks()
+    sweep_p = prefill_sweep(jl, dev, stream, world, rank, 3, bf16_sust)
+    sweep_d = decode_sweep(jl, dev, stream, world, rank, hbm, 50)
+
     # ---------------- end to end through the public API, host buffers ----------
     # Every step copies its inputs from pinned host memory, runs the prefill
     # and the decode through the Python binding, and copies the outputs back.
@@ -432,7 +527,6 @@ def run_cuda(args):
     # pays the write-back of the prefill's output still dirty in L2
     dec_call_ms = max_over_ranks(dec_bif, world)
     dec_gbs = kvb * world / (dec_call_ms / 1e3) / 1e9
-    hbm, bf16_burst, bf16_sust, src = peaks()
     pre_launch_ms = pre_sum / args.steps
     achieved = flops / (pre_launch_ms / 1e3) / 1e12
     line = {
@@ -499,6 +593,8 @@ def run_cuda(args):
             "ms_per_call": round(pre_chunk, 3),
             "tflops": round(chunk_flops * world / (pre_chunk / 1e3) / 1e12, 2),
         },
+        "prefill_sweep": sweep_p,
+        "decode_sweep": sweep_d,
         "prefill": {
             "ms_per_call": round(pre_launch_ms, 3),
             "frac_bf16_sustained": round(achieved / bf16_sust, 4),
@@ -544,7 +640,7 @@ def cpu_baseline(q_h, k_h, v_h, qd_h, kc_h, vc_h, kwp, kwd, pos, budget_s=20.0, 
     orc = oracle.default()
     B, L, Hq, D = q_h.shape
     qa, ka, va = W.to_oracle_array(q_h), W.to_oracle_array(k_h), W.to_oracle_array(v_h)
-    per_head = rows or 8
+    per_head = rows or 16
     rb, rq, rh = W.sample_rows(B, L, Hq, per_head=per_head, seed=123)
     t = time.perf_counter()
     orc.bifocal_rows(qa, ka, va, rb, rq, rh, **kwp)
@@ -578,7 +674,9 @@ def run_reference(args):
     kwp = dict(w_local=pc["w_local"], w_pretrained=pc["w_pretrained"], rope_base=pc["rope_base"])
     q, k, v = W.prefill_inputs(B, L, Hq, Hkv, D, value_scale=pc["value_scale"], seed=pc["seed"])
     qa, ka, va = W.to_oracle_array(q), W.to_oracle_array(k), W.to_oracle_array(v)
-    per_head = 2
+    # the oracle runs the rows of one kv head at a time in parallel: give each
+    # kv head at least as many rows as there are host threads
+    per_head = max(2, -(-orc.num_threads() // (Hq // Hkv)))
     times, flops = [], []
     for s in range(args.warmup + args.steps):
         rb, rq, rh = W.sample_rows(B, L, Hq, per_head=per_head, seed=1000 + s)

@@ -237,7 +237,9 @@ jl_status jl_bifocal_decode(const void *q_new, const void *k_cache_roped,
  *   pos = 131071); larger sizes return JL_ERR_UNSUPPORTED with a message.
  *   The first call on each device looks up that array's device address (with
  *   that device current) and caches it; make that first call before any stream
- *   capture.  Every call shares the array and it keeps the last call's
+ *   capture.  jl_finalize drops the cached addresses: after a device reset
+ *   (cudaDeviceReset), call jl_finalize before the next call, which then looks
+ *   the address up again.  Every call shares the array and it keeps the last call's
  *   partials; each call writes every entry it reads before reading it.  Calls
  *   whose executions overlap on the GPU (other streams, other threads) race on
  *   the array: serialise them.
@@ -321,7 +323,9 @@ const char *jl_last_error(void);
 jl_status jl_check_device_status(jl_stream_t stream);
 
 /* Releases every library-owned device buffer on every device (synchronises
- * each device first).  Later calls re-create them. */
+ * each device first) and forgets the cached device address of
+ * jl_bifocal_decode_noalloc's fixed array.  Later calls re-create them.  Call it
+ * after a device reset, before the library's next call. */
 void jl_finalize(void);
 
 #ifdef __cplusplus

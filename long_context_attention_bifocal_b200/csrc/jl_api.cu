@@ -890,6 +890,7 @@ void jl_finalize(void) {
     d.scratch_bytes = 0;
     d.init = false;
   }
+  decode_noalloc_forget();
   if (have_prev) cudaSetDevice(prev);
 }
 

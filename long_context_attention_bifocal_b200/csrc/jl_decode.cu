@@ -440,13 +440,17 @@ static __device__ __align__(256) float g_decode_noalloc_scratch[kDecodeNoAllocFl
 
 constexpr int kMaxScratchDevices = 64;
 
+std::mutex g_noalloc_mu;
+float *g_noalloc_addr[kMaxScratchDevices] = {};
+
 }  // namespace
 
 // Device address of the fixed scratch array on the current device, resolved
-// once per device (with that device current) and cached.
+// once per device (with that device current) and cached until
+// decode_noalloc_forget().
 cudaError_t decode_noalloc_scratch(float **out) {
-  static std::mutex mu;
-  static float *addr[kMaxScratchDevices] = {};
+  std::mutex &mu = g_noalloc_mu;
+  float **addr = g_noalloc_addr;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -460,6 +464,13 @@ cudaError_t decode_noalloc_scratch(float **out) {
   }
   *out = addr[dev];
   return cudaSuccess;
+}
+
+// Drops the cached addresses (a device reset unloads the module, after which
+// the array may sit elsewhere); the next call on each device resolves it again.
+void decode_noalloc_forget() {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  for (int i = 0; i < kMaxScratchDevices; ++i) g_noalloc_addr[i] = nullptr;
 }
 
 cudaError_t launch_decode_noalloc(const DecodeArgs &a_in, double rope_base, cudaStream_t s) {

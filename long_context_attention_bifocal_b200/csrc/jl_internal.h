@@ -157,5 +157,6 @@ constexpr size_t kDecodeNoAllocFloats = static_cast<size_t>(1) << 20;
 // Same decode, split partials in the library's fixed scratch array and angles
 // evaluated in-kernel; a.ws is ignored.  Allocates nothing.
 cudaError_t launch_decode_noalloc(const DecodeArgs &a, double rope_base, cudaStream_t s);
+void decode_noalloc_forget();
 
 }  // namespace jl

@@ -4,6 +4,7 @@ import pytest
 import torch
 
 import parity
+import prefill_cases as C
 from long_context_attention_bifocal_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -50,28 +51,15 @@ def test_tiny_f32_L128_is_plain_rope(jl, oracle_mod):
 
 
 # ------------------------------------------- bf16, small, every row ----
-SMALL = [
-    # (B, L, Hq, Hkv, w_pretrained, w_local, value_scale)
-    (1, 1000, 4, 2, 300, 200, 0.5),    # G=4, ragged tail, window edge inside a tile
-    (2, 640, 2, 1, 200, 37, 0.5),      # G=4, window narrower than a tile
-    (1, 513, 2, 2, 100, 0, 0.5),       # every pair remote, G=6
-    (1, 700, 2, 1, 100, 5000, 0.5),    # window covers every pair: plain RoPE
-    (1, 1, 1, 1, 10, 2, 0.5),          # one token
-    (1, 129, 2, 1, 64, 128, 0.5),      # G=3, window of exactly one tile
-    (1, 2125, 4, 1, 1024, 256, 0.5),   # GQA 4, G=3
-    (1, 1536, 2, 1, 512, 300, 1.0),    # sharper attention (scores 4x larger)
-    (2, 700, 8, 2, 256, 100, 0.5),     # B=2, two kv heads of two head pairs (CTA order)
-    (1, 600, 6, 2, 200, 64, 0.5),      # GQA 3: odd group, the one-tile kernel
-    (2, 400, 3, 3, 128, 50, 0.5),      # multi-head (group 1), B=2
-    (1, 4096, 2, 1, 16, 100, 0.5),     # G = 256: 256 keys share each remapped position
-]
+# The cases (tests/prefill_cases.py) carry needles: keys planted so that a
+# group size or window edge off by one, or a missing remap, fails the gates
+# (shown on the CPU by test_parity_sensitivity.py).
+SMALL = C.SMALL
 
 
-@pytest.mark.parametrize("case", SMALL, ids=[f"B{c[0]}L{c[1]}H{c[2]}x{c[3]}wp{c[4]}wl{c[5]}s{c[6]}" for c in SMALL])
+@pytest.mark.parametrize("case", SMALL, ids=[C.small_id(c) for c in SMALL])
 def test_bf16_small_all_rows(jl, oracle_mod, case):
-    B, L, Hq, Hkv, wp, wl, sc = case
-    q, k, v = W.prefill_inputs(B, L, Hq, Hkv, 128, dtype="bf16", value_scale=sc, seed=L)
-    kw = dict(w_local=wl, w_pretrained=wp, rope_base=1e6)
+    q, k, v, kw = C.small_inputs(oracle_mod.default(), case)
     out, lse = run_prefill(jl, q, k, v, **kw)
     ref_o, ref_l = oracle_mod.default().bifocal_all_rows(
         W.to_oracle_array(q), W.to_oracle_array(k), W.to_oracle_array(v), **kw)
@@ -79,7 +67,7 @@ def test_bf16_small_all_rows(jl, oracle_mod, case):
                  max_abs=parity.BF16_MAX_ABS, mean_abs=parity.BF16_MEAN_ABS, what=str(case))
 
 
-@pytest.mark.parametrize("case", SMALL, ids=[f"B{c[0]}L{c[1]}H{c[2]}x{c[3]}wp{c[4]}wl{c[5]}s{c[6]}" for c in SMALL])
+@pytest.mark.parametrize("case", SMALL, ids=[C.small_id(c) for c in SMALL])
 def test_bf16_small_all_rows_one_tile_kernel(jl, oracle_mod, case, monkeypatch):
     """The same cases on the one-query-tile kernel (the default takes two query
     heads per CTA whenever the group size is even)."""
@@ -128,8 +116,7 @@ def test_explicit_workspace_matches_library_scratch(jl):
 
 
 # ---------------------------------- full sizes, sampled rows per head ----
-FULL = ["qwen3_1p7b_L65536", "qwen3_8b_L131072", "qwen3_4b_L16384", "qwen3_4b_L32768",
-        "qwen3_4b_L49152", "qwen3_4b_L98304", "qwen3_4b_L131072"]
+FULL = C.FULL
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -143,17 +130,15 @@ def test_full_size_sampled_rows_one_tile_kernel(jl, oracle_mod, monkeypatch):
 
 
 def full_size_sampled_rows(jl, oracle_mod, name):
+    """The configuration's own inputs, 512 seeded rows per head plus the rows at
+    the window edge, tile and group boundaries and the ends."""
     cfg = W.PREFILL[name]
-    B, L, Hq, Hkv, D = cfg["B"], cfg["L"], cfg["Hq"], cfg["Hkv"], cfg["D"]
-    q, k, v = W.prefill_inputs(B, L, Hq, Hkv, D, value_scale=cfg["value_scale"],
-                               seed=cfg["seed"])
-    kw = params(cfg)
+    B, L, Hq = cfg["B"], cfg["L"], cfg["Hq"]
+    q, k, v, kw = C.full_inputs(name)
     out, lse = run_prefill(jl, q, k, v, **kw)
     G = oracle_mod.default().group_size(L, cfg["w_pretrained"])
-    wl = cfg["w_local"]
-    extra = [0, 1, 127, 128, wl - 1, wl, wl + 1, L // 2, L - 2, L - 1]
-    extra += [G * m for m in (1, 1000)] + [G * m - 1 for m in (1, 1000)]
-    rb, rq, rh = W.sample_rows(B, L, Hq, per_head=512, seed=cfg["seed"], extra=extra)
+    rb, rq, rh = W.sample_rows(B, L, Hq, per_head=512, seed=cfg["seed"],
+                               extra=C.edge_positions(L, G, cfg["w_local"]))
     ref_o, ref_l = oracle_mod.default().bifocal_rows(
         W.to_oracle_array(q), W.to_oracle_array(k), W.to_oracle_array(v), rb, rq, rh, **kw)
     go, gl = parity.gather_rows(out, lse, rb, rq, rh)
@@ -163,3 +148,55 @@ def full_size_sampled_rows(jl, oracle_mod, name):
     if G == 1:
         out0, lse0 = run_prefill(jl, q, k, v, flags=jl.NO_BIFOCAL, **kw)
         assert torch.equal(out, out0) and torch.equal(lse, lse0)
+
+
+def needle_case(jl, oracle_mod, name, qk_scale=None):
+    """Full-size inputs with needles: the needle rows (each dominated by one
+    key whose score is right only under the bifocal rule) and 16 seeded rows
+    per head.  Besides the gates, the output must be far from the same
+    kernel's plain-RoPE output (JL_FLAG_NO_BIFOCAL) wherever the two rules
+    differ: at least ten times farther than it is from the oracle."""
+    orc = oracle_mod.default()
+    cfg = W.PREFILL[name]
+    B, L, Hq = cfg["B"], cfg["L"], cfg["Hq"]
+    q, k, v, kw, nd = C.needle_inputs(orc, name, qk_scale=qk_scale)
+    out, lse = run_prefill(jl, q, k, v, **kw)
+    rb, rq, rh = C.needle_rows(nd, B, L, Hq, per_head=16, seed=cfg["seed"])
+    ref_o, ref_l = orc.bifocal_rows(
+        W.to_oracle_array(q), W.to_oracle_array(k), W.to_oracle_array(v), rb, rq, rh, **kw)
+    go, gl = parity.gather_rows(out, lse, rb, rq, rh)
+    stats = parity.check(go, gl, ref_o, ref_l, max_abs=parity.BF16_MAX_ABS,
+                         mean_abs=parity.BF16_MEAN_ABS, what=f"{name} needles")
+    n = len(nd)
+    row_rel = (np.abs(go[:n] - ref_o[:n]).max(axis=1) /
+               np.maximum(np.abs(ref_o[:n]).max(axis=1), 1e-30))
+    print(name, "needles", n, stats, "needle-row relative max", float(row_rel.max()))
+    assert row_rel.max() <= 0.05, f"{name}: needle-row relative error {row_rel.max():.3e}"
+    G = orc.group_size(L, cfg["w_pretrained"])
+    if G > 1:
+        out0, lse0 = run_prefill(jl, q, k, v, flags=jl.NO_BIFOCAL, **kw)
+        po, _ = parity.gather_rows(out0, lse0, rb, rq, rh)
+        remote = np.array([x[2] - x[3] >= kw["w_local"] for x in nd])
+        err = np.abs(go[:n] - ref_o[:n]).max(axis=1)[remote]
+        dist = np.abs(go[:n] - po[:n]).max(axis=1)[remote]
+        print(name, "distance to plain RoPE on remote needle rows: min", float(dist.min()),
+              "error against the oracle: max", float(err.max()))
+        assert dist.min() > 10 * err.max()
+    return stats
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_needles(jl, oracle_mod, name):
+    needle_case(jl, oracle_mod, name)
+
+
+@pytest.mark.parametrize("name", sorted(C.PEAKY))
+def test_full_size_peaky(jl, oracle_mod, name):
+    """q and k at four times the configurations' scale (scores with a standard
+    deviation of ~4: a few dozen keys carry each row) plus needles."""
+    needle_case(jl, oracle_mod, name, qk_scale=C.PEAKY[name])
+
+
+def test_full_size_needles_one_tile_kernel(jl, oracle_mod, monkeypatch):
+    monkeypatch.setenv("JL_PREFILL_KERNEL", "one")
+    needle_case(jl, oracle_mod, "qwen3_8b_L131072")
