@@ -23,7 +23,9 @@
  *   - Softmax scale defaults to 1/sqrt(D).  lse is the natural log of
  *     sum_k exp(scale * score_k), in fp32.
  *   - All tensor pointers are caller-owned DEVICE memory, contiguous, 16-byte
- *     aligned.  The library writes only `out`, `lse` and the workspace.
+ *     aligned.  The library writes only `out`, `lse` and the workspace (the
+ *     decode and the three-call prefill take one; the fused prefill and the
+ *     chunked prefill rotate their keys inside the kernels and need none).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream).  No entry point synchronises the host with the device except the
  *     first call that builds or grows a library-owned table (see below) and
@@ -34,14 +36,12 @@
  *     and no kernel traps.
  *   - Library-owned device memory: per device, a cos/sin table of the RoPE
  *     angles (fp64 sincos rounded to fp32, [positions][D/2] pairs) grown on
- *     demand, a 4-byte device status word, and a grown scratch buffer for the
- *     prefill calls given no workspace.  A table or scratch buffer that is
- *     replaced by a larger one stays allocated (launches in flight may read
- *     it) until jl_finalize, which releases them all.  The first call that
- *     creates or grows them allocates and synchronises its stream, so make it
- *     before any stream capture.  Prefill calls that use the library's scratch
- *     buffer and overlap on the GPU (other streams, other threads) race on it:
- *     serialise them, or give each its own workspace (jl_bifocal_prefill_ex).
+ *     demand, and a 4-byte device status word.  A table that is replaced by a
+ *     larger one stays allocated (launches in flight may read it) until
+ *     jl_finalize, which releases them all.  The first call that creates or
+ *     grows the table allocates and synchronises its stream, so make it before
+ *     any stream capture.  The library holds no per-call scratch: calls on
+ *     different streams may overlap on the GPU.
  */
 #ifndef JETLONG_H
 #define JETLONG_H
@@ -106,15 +106,18 @@ long long jl_group_size(long long L, long long w_pretrained);
  *   out  [B, L, Hq, D]  bf16 (written)
  *   lse  [B, Hq, L]     fp32 (written)
  *   D == 128.  w_local >= 0 (0 = every pair remote), w_pretrained >= 1,
- *   rope_base > 1.  The library's scratch buffer holds the rotated keys
- *   (2 * B * L * Hkv * D bf16); it is grown on demand.
+ *   rope_base > 1.  Queries and keys are rotated inside the attention kernel
+ *   (keys tile by tile in shared memory, to R(k) for the local passes and to
+ *   R(f(k)) for the remote ones), so the call needs no memory beyond its
+ *   arguments.
  */
 jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v,
                              void *out, float *lse, int B, int L, int Hq,
                              int Hkv, int D, int w_local, int w_pretrained,
                              double rope_base, jl_stream_t stream);
 
-/* Bytes of caller workspace jl_bifocal_prefill_ex needs (0 for fp32). */
+/* Bytes of caller workspace jl_bifocal_prefill_ex needs: 0 for every size and
+ * dtype (the keys are rotated inside the kernels). */
 size_t jl_bifocal_prefill_workspace_size(int B, int L, int Hkv, int D,
                                          jl_dtype dtype);
 
@@ -122,8 +125,8 @@ size_t jl_bifocal_prefill_workspace_size(int B, int L, int Hkv, int D,
  * Bifocal prefill with every option.  dtype JL_BF16 (D == 128, tensor cores)
  * or JL_F32 (D in {64, 128}, fp32 CUDA-core kernel; out is fp32).
  * softmax_scale <= 0 selects 1/sqrt(D).  flags: JL_FLAG_NO_BIFOCAL.
- * workspace: device memory of at least jl_bifocal_prefill_workspace_size()
- * bytes, 256-byte aligned; NULL selects the library-owned buffer.
+ * workspace, workspace_bytes: not used (no workspace is needed); any value,
+ * NULL and 0 included, is accepted and nothing is written there.
  */
 jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v,
                                 void *out, float *lse, int B, int L, int Hq,
@@ -175,11 +178,12 @@ jl_status jl_bifocal_prefill_3pass(const void *q, const void *k, const void *v,
  * the local/remote rule of jl_bifocal_prefill over keys [0, q_offset + Lq): the
  * result is rows q_offset .. q_offset + Lq - 1 of jl_bifocal_prefill over the
  * whole sequence (up to the bf16 rounding of the cached keys).  Keys at
- * remapped positions are formed from the cache as R(f(k) - k) k_cache.
+ * remapped positions are formed from the cache as R(f(k) - k) k_cache, tile by
+ * tile inside the kernel; the cache is only read.
  * q_offset a multiple of 128 (JL_ERR_UNSUPPORTED otherwise), q_offset + Lq <=
  * cache_capacity, D == 128, flags: JL_FLAG_NO_BIFOCAL.
- * workspace: at least jl_bifocal_prefill_chunk_workspace_size() bytes,
- * 256-byte aligned (the remapped keys); NULL selects the library's scratch.
+ * workspace, workspace_bytes: not used (no workspace is needed; the size
+ * query returns 0); any value, NULL and 0 included, is accepted.
  */
 size_t jl_bifocal_prefill_chunk_workspace_size(int B, int q_offset, int Lq, int Hkv,
                                                int D);

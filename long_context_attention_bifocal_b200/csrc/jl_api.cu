@@ -36,9 +36,7 @@ struct DeviceState {
   int table_D = 0;
   double table_base = 0.0;
   unsigned *status = nullptr;
-  void *scratch = nullptr;
-  size_t scratch_bytes = 0;
-  // buffers replaced by larger ones: another host thread may hold a pointer
+  // tables replaced by larger ones: another host thread may hold a pointer
   // to one between taking it and launching, so they live until jl_finalize
   std::vector<void *> retired;
 };
@@ -148,38 +146,11 @@ jl_status status_word(unsigned **out) {
   return JL_OK;
 }
 
-jl_status prefill_scratch(size_t bytes, void **out) {
-  DeviceState *d = nullptr;
-  jl_status st = current(&d);
-  if (st != JL_OK) return st;
-  std::lock_guard<std::mutex> lock(d->mu);
-  if (d->scratch_bytes < bytes) {
-    if (d->scratch) {  // kept alive, as the tables are
-      d->retired.push_back(d->scratch);
-      d->scratch = nullptr;
-      d->scratch_bytes = 0;
-    }
-    void *p = nullptr;
-    cudaError_t e = cudaMalloc(&p, bytes);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(prefill scratch)");
-    d->scratch = p;
-    d->scratch_bytes = bytes;
-  }
-  *out = d->scratch;
-  return JL_OK;
-}
-
 }  // namespace jl
 
 using namespace jl;
 
 namespace {
-
-size_t prefill_ws_bytes(int B, int L, int Hkv, int D) {
-  const size_t one = static_cast<size_t>(B) * L * Hkv * D * sizeof(__nv_bfloat16);
-  const size_t aligned = (one + 255) & ~static_cast<size_t>(255);
-  return 2 * aligned;  // rotated keys at original and at remapped positions
-}
 
 jl_status check_common(int B, int L, int Hq, int Hkv, int D, int w_local, int w_pretrained,
                        double rope_base) {
@@ -217,9 +188,9 @@ long long jl_group_size(long long L, long long w_pretrained) {
 const char *jl_last_error(void) { return g_last_error.c_str(); }
 
 size_t jl_bifocal_prefill_workspace_size(int B, int L, int Hkv, int D, jl_dtype dtype) {
-  if (B < 1 || L < 1 || Hkv < 1 || D < 1) return 0;
-  if (dtype != JL_BF16) return 0;
-  return prefill_ws_bytes(B, L, Hkv, D);
+  // keys are rotated inside the prefill kernels: no workspace for any size
+  (void)B, (void)L, (void)Hkv, (void)D, (void)dtype;
+  return 0;
 }
 
 jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v, void *out,
@@ -247,14 +218,7 @@ jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v, voi
     return fail(JL_ERR_UNSUPPORTED, "problem too large for one launch");
   if (!(softmax_scale >= 0.f) && !(softmax_scale < 0.f))
     return fail(JL_ERR_INVALID_ARG, "softmax_scale is NaN");
-  const size_t need_ws = dtype == JL_BF16 ? prefill_ws_bytes(B, L, Hkv, D) : 0;
-  if (workspace != nullptr) {
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-      return fail(JL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-    if (workspace_bytes < need_ws)
-      return fail(JL_ERR_INVALID_ARG, "workspace too small: %zu bytes, need %zu",
-                  workspace_bytes, need_ws);
-  }
+  (void)workspace, (void)workspace_bytes;  // unused: keys are rotated in the kernels
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const long long G = group_size_ll(L, w_pretrained);
@@ -273,7 +237,7 @@ jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v, voi
   a.G = static_cast<int>(G);
   a.w_eff = plain ? INT_MAX : w_local;
   a.scale = softmax_scale > 0.f ? softmax_scale : static_cast<float>(1.0 / std::sqrt(D));
-  a.kstd = a.krem = nullptr;
+  a.key_mode = 0;  // raw keys, rotated in the kernel
   st = rope_table(D, rope_base, L, s, &a.table);
   if (st != JL_OK) return st;
   st = status_word(&a.status);
@@ -284,24 +248,7 @@ jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v, voi
     return e == cudaSuccess ? JL_OK : cuda_fail(e, "fp32 prefill launch");
   }
 
-  void *ws = workspace;
-  if (ws == nullptr) {
-    st = prefill_scratch(need_ws, &ws);
-    if (st != JL_OK) return st;
-  }
-  const size_t one = need_ws / 2;
-  __nv_bfloat16 *kstd = static_cast<__nv_bfloat16 *>(ws);
-  __nv_bfloat16 *krem =
-      reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + one);
-  const bool need_std = a.w_eff > 0;
-  const bool need_rem = !plain;  // some pair is remote
-  cudaError_t e = launch_rotate_keys(static_cast<const __nv_bfloat16 *>(k),
-                                     need_std ? kstd : nullptr, need_rem ? krem : nullptr,
-                                     a.table, B, L, Hkv, D, a.G, s);
-  if (e != cudaSuccess) return cuda_fail(e, "key rotation launch");
-  a.kstd = need_std ? kstd : nullptr;
-  a.krem = need_rem ? krem : nullptr;
-  e = launch_attention(a, s);
+  cudaError_t e = launch_attention(a, s);
   return e == cudaSuccess ? JL_OK : cuda_fail(e, "prefill launch");
 }
 
@@ -313,10 +260,9 @@ jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v, void *
 }
 
 size_t jl_bifocal_prefill_chunk_workspace_size(int B, int q_offset, int Lq, int Hkv, int D) {
-  if (B < 1 || q_offset < 0 || Lq < 1 || Hkv < 1 || D < 2) return 0;
-  const size_t one =
-      static_cast<size_t>(B) * (static_cast<size_t>(q_offset) + Lq) * Hkv * D * sizeof(__nv_bfloat16);
-  return (one + 255) & ~static_cast<size_t>(255);
+  // the remote passes correct the cached keys inside the kernels: no workspace
+  (void)B, (void)q_offset, (void)Lq, (void)Hkv, (void)D;
+  return 0;
 }
 
 jl_status jl_bifocal_prefill_chunk(const void *q, const void *k_cache_roped, const void *v_cache,
@@ -345,14 +291,7 @@ jl_status jl_bifocal_prefill_chunk(const void *q, const void *k_cache_roped, con
   if (Lk >= (1LL << 31) - 256) return fail(JL_ERR_UNSUPPORTED, "sequence too long");
   if (static_cast<long long>((Lq + 127) / 128) * B * Hq >= (1LL << 31))
     return fail(JL_ERR_UNSUPPORTED, "problem too large for one launch");
-  const size_t need = jl_bifocal_prefill_chunk_workspace_size(B, q_offset, Lq, Hkv, D);
-  if (workspace != nullptr) {
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-      return fail(JL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-    if (workspace_bytes < need)
-      return fail(JL_ERR_INVALID_ARG, "workspace too small: %zu bytes, need %zu",
-                  workspace_bytes, need);
-  }
+  (void)workspace, (void)workspace_bytes;  // unused: keys are corrected in the kernels
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const long long G = group_size_ll(Lk, w_pretrained);
@@ -376,22 +315,10 @@ jl_status jl_bifocal_prefill_chunk(const void *q, const void *k_cache_roped, con
   if (st != JL_OK) return st;
   st = status_word(&a.status);
   if (st != JL_OK) return st;
-  // keys at original positions: the cache itself; at remapped positions: a
-  // compact corrected copy in the workspace
-  a.kstd = a.w_eff > 0 ? k_cache_roped : nullptr;
-  a.krem = nullptr;
-  if (!plain) {
-    void *ws = workspace;
-    if (ws == nullptr) {
-      st = prefill_scratch(need, &ws);
-      if (st != JL_OK) return st;
-    }
-    cudaError_t e = launch_correct_keys(static_cast<const __nv_bfloat16 *>(k_cache_roped),
-                                        static_cast<__nv_bfloat16 *>(ws), a.table, B,
-                                        static_cast<int>(Lk), cache_capacity, Hkv, D, a.G, s);
-    if (e != cudaSuccess) return cuda_fail(e, "key correction launch");
-    a.krem = ws;
-  }
+  // keys at original positions: the cache as it is; at remapped positions:
+  // R(f(k) - k) of the cached key, applied in the kernel
+  a.k = k_cache_roped;
+  a.key_mode = 1;
   cudaError_t e = launch_attention(a, s);
   return e == cudaSuccess ? JL_OK : cuda_fail(e, "chunked prefill launch");
 }
@@ -401,7 +328,7 @@ size_t jl_bifocal_prefill_3pass_workspace_size(int B, int L, int Hq, int Hkv, in
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   const size_t o = up(static_cast<size_t>(B) * L * Hq * D * sizeof(__nv_bfloat16));
   const size_t l = up(static_cast<size_t>(B) * Hq * L * sizeof(float));
-  return prefill_ws_bytes(B, L, Hkv, D) + 2 * o + 2 * l;
+  return 2 * o + 2 * l;
 }
 
 jl_status jl_bifocal_prefill_3pass(const void *q, const void *k, const void *v, void *out,
@@ -447,9 +374,7 @@ jl_status jl_bifocal_prefill_3pass(const void *q, const void *k, const void *v, 
 
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   char *ws = static_cast<char *>(workspace);
-  const size_t kb = prefill_ws_bytes(B, L, Hkv, D);
-  __nv_bfloat16 *kstd = reinterpret_cast<__nv_bfloat16 *>(ws);
-  __nv_bfloat16 *krem = reinterpret_cast<__nv_bfloat16 *>(ws + kb / 2);
+  const size_t kb = 0;
   const size_t ob = up(static_cast<size_t>(B) * L * Hq * D * sizeof(__nv_bfloat16));
   const size_t lb = up(static_cast<size_t>(B) * Hq * L * sizeof(float));
   __nv_bfloat16 *o_b = reinterpret_cast<__nv_bfloat16 *>(ws + kb);
@@ -457,31 +382,23 @@ jl_status jl_bifocal_prefill_3pass(const void *q, const void *k, const void *v, 
   float *l_b = reinterpret_cast<float *>(ws + kb + 2 * ob);
   float *l_c = reinterpret_cast<float *>(ws + kb + 2 * ob + lb);
 
-  cudaError_t e = launch_rotate_keys(static_cast<const __nv_bfloat16 *>(k),
-                                     w_local > 0 ? kstd : nullptr, krem, a.table, B, L, Hkv, D,
-                                     a.G, s);
-  if (e != cudaSuccess) return cuda_fail(e, "key rotation launch");
   // A: every pair at remapped positions, into out / lse
+  a.k = k;
+  a.key_mode = 0;
   a.out = out;
   a.lse = lse;
-  a.kstd = nullptr;
-  a.krem = krem;
   a.w_eff = 0;
   a.band = 0;
-  e = launch_attention(a, s);
+  cudaError_t e = launch_attention(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch (A)");
   if (w_local == 0) return JL_OK;  // empty window: B and C have no pairs
   // B: the local window at original positions; C: the same window remapped
   a.w_eff = w_local;
-  a.kstd = kstd;
-  a.krem = nullptr;
   a.band = 1;
   a.out = o_b;
   a.lse = l_b;
   e = launch_attention(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch (B)");
-  a.kstd = nullptr;
-  a.krem = krem;
   a.band = 2;
   a.out = o_c;
   a.lse = l_c;
@@ -880,14 +797,11 @@ void jl_finalize(void) {
     cudaDeviceSynchronize();
     if (d.table) cudaFree(d.table);
     if (d.status) cudaFree(d.status);
-    if (d.scratch) cudaFree(d.scratch);
     for (void *r : d.retired) cudaFree(r);
     d.retired.clear();
     d.table = nullptr;
     d.status = nullptr;
-    d.scratch = nullptr;
     d.table_positions = 0;
-    d.scratch_bytes = 0;
     d.init = false;
   }
   decode_noalloc_forget();

@@ -33,29 +33,15 @@ jl_status cuda_fail(cudaError_t e, const char *what);
 jl_status rope_table(int D, double base, int min_positions, cudaStream_t s,
                      RopeTable *out);
 jl_status status_word(unsigned **out);
-jl_status prefill_scratch(size_t bytes, void **out);
 int sm_count();
 
 // ---- launchers (each returns the launch's cudaError_t) ----
 cudaError_t launch_rope_table(float2 *cs, int positions, int D, double base, cudaStream_t s);
 
-// Keys [0, L) of a cache [B, cap, Hkv, D] rotated at their original positions,
-// moved to remapped positions: krem[b, k] = R(f(k) - k) kc[b, k], written
-// compactly as [B, L, Hkv, D].
-cudaError_t launch_correct_keys(const __nv_bfloat16 *kc, __nv_bfloat16 *krem, RopeTable t,
-                                int B, int L, int cap, int Hkv, int D, int G, cudaStream_t s);
-
-// Rotated copies of the keys of a [B,L,Hkv,D] bf16 tensor:
-// kstd = R(l) k (if kstd), krem = R(floor(l/G)) k (if krem).
-cudaError_t launch_rotate_keys(const __nv_bfloat16 *k, __nv_bfloat16 *kstd,
-                               __nv_bfloat16 *krem, RopeTable t, int B, int L,
-                               int Hkv, int D, int G, cudaStream_t s);
-
 struct PrefillArgs {
   const void *q;      // [B,L,Hq,D] pre-RoPE
-  const void *kstd;   // [B,L,Hkv,D] keys rotated at original positions (bf16 path)
-  const void *krem;   // [B,L,Hkv,D] keys rotated at floor(l/G)         (bf16 path)
-  const void *k;      // raw keys (fp32 path)
+  const void *k;      // [B,L,Hkv,D] keys: raw (key_mode 0) or a cache rotated at
+                      // original positions (key_mode 1, batch stride kv_stride)
   const void *v;      // [B,L,Hkv,D]
   void *out;          // [B,L,Hq,D]
   float *lse;         // [B,Hq,L]
@@ -67,7 +53,9 @@ struct PrefillArgs {
   unsigned *status;
   int band = 0;       // 0: bifocal rule; 1 / 2: only the local window, standard / remapped
   int q_off = 0;      // position of query row 0 (multiple of 128); keys are [0, q_off + L)
-  int64_t kv_stride = 0;  // keys per batch entry in v (and a cache-resident kstd); 0: q_off + L
+  int64_t kv_stride = 0;  // keys per batch entry in k and v; 0: q_off + L
+  int key_mode = 0;   // 0: raw keys (R(k) / R(f(k)) in the kernel); 1: cached keys at
+                      // original positions (as they are / R(f(k) - k) in the kernel)
 };
 
 cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s);

@@ -125,6 +125,61 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8]) {
   }
 }
 
+// Where the keys come from: raw (pre-RoPE) keys, rotated here to R(k) for the
+// local passes and to R(f(k)) for the remote ones; or a cache whose keys are
+// already rotated at their original positions, used as they are by the local
+// passes and moved to f(k) by R(f(k) - k) for the remote ones (techwalker
+// explainer §三: rotations compose, R(a) R(b) = R(a + b)).
+enum : int { kKeysRaw = 0, kKeysCached = 1 };
+
+// Rotates a 128-key tile in shared memory, in place, for a pass of class
+// `kind` (kStd / kRem) over keys k0 .. k0 + 127, bf16 in the 128-byte-swizzled
+// K-major layout the TMA wrote: dims 0-63 in the first 16 KB half, 64-127 in
+// the second, pair (i, i + 64) at the same offset of the two halves.  The
+// `nthr` threads calling it (thread index `tid`) split the 128 x 8 chunks of
+// eight pairs between them; a thread's lanes of one warp take four rows of
+// eight chunks, so table reads and shared-memory accesses stay contiguous.
+// Rows at or past n_keys (zero fill beyond the sequence) are left alone.
+// Arithmetic: fp32 with the fp32 table value of (cos, sin)(p theta_i), one
+// rounding to bf16 at the end.
+__device__ __forceinline__ void rotate_k_tile(uint8_t *tile, int k0, int kind, int key_mode,
+                                              int G, int n_keys, const float2 *cs, int tid,
+                                              int nthr) {
+  if (key_mode == kKeysCached && kind == kStd) return;  // already at original positions
+#pragma unroll 1
+  for (int item = tid; item < kBN * 8; item += nthr) {
+    const int r = item >> 3, c = item & 7;
+    const int k = k0 + r;
+    if (k >= n_keys) continue;
+    int p;
+    float sgn = 1.f;
+    if (key_mode == kKeysRaw) {
+      p = kind == kStd ? k : k / G;
+    } else {
+      p = k - k / G;  // R(f(k) - k) = R(-u): the table row u with the sine negated
+      sgn = -1.f;
+    }
+    uint4 *a1 = reinterpret_cast<uint4 *>(tile + swz(r, c));
+    uint4 *a2 = reinterpret_cast<uint4 *>(tile + kHalfBytes + swz(r, c));
+    float x1[8], x2[8];
+    unpack8(*a1, x1);
+    unpack8(*a2, x2);
+    const float4 *t = reinterpret_cast<const float4 *>(cs + static_cast<int64_t>(p) * 64 + 8 * c);
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float4 r2 = __ldg(t + e);  // (cos, sin) of pairs 2e and 2e + 1
+      const float s0 = sgn * r2.y, s1 = sgn * r2.w;
+      lo[e] = pack_bf16x2(x1[2 * e] * r2.x - x2[2 * e] * s0,
+                          x1[2 * e + 1] * r2.z - x2[2 * e + 1] * s1);
+      hi[e] = pack_bf16x2(x1[2 * e] * s0 + x2[2 * e] * r2.x,
+                          x1[2 * e + 1] * s1 + x2[2 * e + 1] * r2.z);
+    }
+    *a1 = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *a2 = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  }
+}
+
 // 2^x on the FMA/ALU pipes instead of the MUFU unit, for x <= 8:
 // 2^floor(x) * p(x - floor(x)) with a cubic p fitted by weighted least squares
 // on Chebyshev nodes with p(0) = 1 and p(1) = 2 (derive_exp2_poly.py; maximum

@@ -29,11 +29,13 @@
 //              each row's exponentials run on the FMA pipe (exp2_poly).
 //              With P double-buffered the softmax of pass j+1 overlaps the
 //              product O += P V of pass j.
-//   warp 4     TMA producer: K tile (pre-rotated copy of the needed class) and
-//              V tile per pass into a 2-stage ring.
+//   warp 4     TMA producer: raw K tile and V tile per pass into a 3-stage ring.
 //   warp 5     allocates TMEM and issues every tcgen05.mma from one thread:
 //              S = Q K^T (M=N=128, K=128: 8 x K16 steps) into one of two TMEM
 //              S buffers, and O += P V into the TMEM O accumulator.
+//   warps 6-7  rotate each K tile in shared memory, in place, to the pass's
+//              positions (R(k) or R(f(k)) from the cos/sin table) before the
+//              score product reads it: RoPE applied on the fly.
 // Every mbarrier wait is bounded (1 s); a thread that gives up raises the
 // CTA's abort flag and the device status word, after which all CTAs drain and
 // return without touching their outputs further.
@@ -53,7 +55,9 @@ using namespace prefill;
 
 // shared-memory layout (bytes from the 1 KiB-aligned base), barriers, TMEM
 constexpr int kStages = 3;
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;
+constexpr int kRotWarp0 = 6;  // warps 6 and 7 rotate the K tiles
+constexpr int kRotThreads = 64;
 
 constexpr uint32_t kOffQ = 0;  // the Q variant of the current phase
 constexpr uint32_t kOffK = kOffQ + kTileBytes;
@@ -66,7 +70,8 @@ enum : int {
   kBarKEmpty = kBarKFull + kStages,
   kBarVFull = kBarKEmpty + kStages,
   kBarVEmpty = kBarVFull + kStages,
-  kBarSFull = kBarVEmpty + kStages,
+  kBarKRot = kBarVEmpty + kStages,  // [kStages] K tile rotated, kRotThreads arrivals
+  kBarSFull = kBarKRot + kStages,
   kBarSFree = kBarSFull + 2,
   kBarPFull = kBarSFree + 2,  // [2] per P buffer
   kBarODone = kBarPFull + 2,  // [2] per P buffer: O += P V of that buffer done
@@ -102,6 +107,8 @@ struct KParams {
   int B, L, Hq, Hkv, G, w, n_qtiles;
   int band;   // kBandNone, kBandStd or kBandRem
   int q_off;  // position of query row 0 (a multiple of 128; keys start at 0)
+  int key_mode;  // kKeysRaw or kKeysCached
+  int n_keys;    // keys [0, n_keys) exist (q_off + L)
   float scale_log2;  // softmax scale * log2(e)
 };
 
@@ -109,8 +116,7 @@ struct KParams {
 // chunked prefill); the default prefill runs the instantiation without them.
 template <bool kGeneral>
 __global__ void __launch_bounds__(kThreads, 1)
-    bifocal_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_kstd,
-                                 const __grid_constant__ CUtensorMap tm_krem,
+    bifocal_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_k,
                                  const __grid_constant__ CUtensorMap tm_v,
                                  const KParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -147,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarKEmpty + s), 1);
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarVEmpty + s), 1);
+      mbar_init(bar(kBarKRot + s), kRotThreads);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarSFull + s), 1);
@@ -380,8 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 4) {
       // ------------------------------------------------------ TMA producer --
       if (lane == 0) {
-        prefetch_tmap(&tm_kstd);
-        prefetch_tmap(&tm_krem);
+        prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
         PassIter t;
         t.begin(qt + q_off / kBM, p.w, band);
@@ -393,10 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             raise_abort(abort_s, p.status);
             break;
           }
-          const CUtensorMap *km = t.kind() == kStd ? &tm_kstd : &tm_krem;
           mbar_arrive_expect_tx(bar(kBarKFull + s), kTileBytes);
-          tma_load_4d(sb + kOffK + s * kTileBytes, km, bar(kBarKFull + s), 0, hk, kBN * t.j, b);
-          tma_load_4d(sb + kOffK + s * kTileBytes + kHalfBytes, km, bar(kBarKFull + s), 64, hk,
+          tma_load_4d(sb + kOffK + s * kTileBytes, &tm_k, bar(kBarKFull + s), 0, hk, kBN * t.j, b);
+          tma_load_4d(sb + kOffK + s * kTileBytes + kHalfBytes, &tm_k, bar(kBarKFull + s), 64, hk,
                       kBN * t.j, b);
           ++kiss;
           if (!mbar_wait(bar(kBarVEmpty + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
@@ -417,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           drain_wait(bar(kBarVFull + d % kStages), (d / kStages) & 1);
       }
       __syncwarp();
-    } else {
+    } else if (warp == 5) {
       // ------------------------------------------------------- MMA issuer --
       if (lane == 0) {
         const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
@@ -459,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ph = (it / kStages) & 1;
           const int sbuf = it & 1;
           const uint32_t sph = (it >> 1) & 1;
-          if (!mbar_wait(bar(kBarKFull + s), ph, abort_s, abort_g, kTimeoutNs) ||
+          if (!mbar_wait(bar(kBarKRot + s), ph, abort_s, abort_g, kTimeoutNs) ||
               !mbar_wait(bar(kBarSFree + sbuf), sph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
             ok = false;
             break;
@@ -490,6 +495,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(bar(kBarDrain), 0);
       }
       __syncwarp();
+    } else {
+      // --------------------------------------------------- K rotation (6-7) --
+      // Pass n's K tile sits in stage n % kStages; once the TMA has landed it,
+      // it is rotated in place to its pass's positions and handed to the MMA
+      // warp (kBarKRot).  The producer refills a stage only after the score
+      // product has read it.
+      const int tid = static_cast<int>(threadIdx.x) - 32 * kRotWarp0;
+      PassIter t;
+      t.begin(qt + q_off / kBM, p.w, band);
+      int n = 0;
+      while (!t.done()) {
+        const int s = n % kStages;
+        if (!mbar_wait(bar(kBarKFull + s), (n / kStages) & 1, abort_s, abort_g, kTimeoutNs)) {
+          raise_abort(abort_s, p.status);
+          break;
+        }
+        rotate_k_tile(smem + kOffK + s * kTileBytes, kBN * t.j, t.kind(), p.key_mode, p.G,
+                      p.n_keys, p.cs, tid, kRotThreads);
+        fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
+        mbar_arrive(bar(kBarKRot + s));
+        ++n;
+        t.next();
+      }
     }
   }
   __syncthreads();
@@ -544,16 +572,12 @@ cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s) {
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  CUtensorMap mks, mkr, mv;
-  const void *krem = a.krem ? a.krem : a.kstd;
-  const void *kstd = a.kstd ? a.kstd : a.krem;
-  // keys [0, q_off + L); the cache-resident tensors (K_std, V) may be longer
-  // per batch entry than that (kv_stride keys)
+  CUtensorMap mk, mv;
+  // keys [0, q_off + L); a cache may be longer per batch entry than that
+  // (kv_stride keys)
   const int keys = a.q_off + a.L;
   const int64_t kvs = a.kv_stride > 0 ? a.kv_stride : keys;
-  if (!make_map(&mks, kstd, a.B, keys, a.Hkv, a.kstd ? kvs : keys) ||
-      !make_map(&mkr, krem, a.B, keys, a.Hkv, a.krem ? keys : kvs) ||
-      !make_map(&mv, a.v, a.B, keys, a.Hkv, kvs))
+  if (!make_map(&mk, a.k, a.B, keys, a.Hkv, kvs) || !make_map(&mv, a.v, a.B, keys, a.Hkv, kvs))
     return cudaErrorInvalidValue;
   KParams p;
   p.q = static_cast<const __nv_bfloat16 *>(a.q);
@@ -569,13 +593,15 @@ cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s) {
   p.w = a.w_eff;
   p.band = a.band;
   p.q_off = a.q_off;
+  p.key_mode = a.key_mode;
+  p.n_keys = keys;
   p.n_qtiles = (a.L + kBM - 1) / kBM;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * a.Hq;
   if (a.band != 0 || a.q_off != 0)
-    bifocal_prefill_sm100_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mks, mkr, mv, p);
+    bifocal_prefill_sm100_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mv, p);
   else
-    bifocal_prefill_sm100_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mks, mkr, mv, p);
+    bifocal_prefill_sm100_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mv, p);
   return cudaGetLastError();
 }
 

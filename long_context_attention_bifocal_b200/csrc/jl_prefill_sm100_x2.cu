@@ -12,10 +12,12 @@
 // Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax of head 0: thread r = query row r = TMEM lane r of S0/O0
 //   warps 4-7  softmax of head 1: the same on S1/O1
-//   warp 8     TMA producer: K tile (pre-rotated copy of the pass's class) and
-//              V tile into a 2-stage ring
+//   warp 8     TMA producer: raw K tile and V tile into a 2-stage ring
 //   warp 9     TMEM allocation and every tcgen05.mma, from one thread
-//   warps 10-11 idle (they complete the third warpgroup)
+//   warps 10-11 rotate each K tile in shared memory, in place, to the pass's
+//              positions (R(k) or R(f(k)) from the cos/sin table) before the
+//              score product reads it: RoPE applied on the fly, with no
+//              rotated copy of the keys in global memory
 // Registers: launched at 168 a thread; the third warpgroup drops to 72 and the
 // softmax warpgroups rise to 216 (setmaxnreg), so a softmax thread holds its
 // whole S row and reads S from TMEM once per pass.
@@ -32,7 +34,7 @@
 // tile all come before its local passes, so Q_rem is used first and is then
 // overwritten in place by Q_std (one switch per tile, signalled through the
 // q_ready barrier).  Q rotation runs in the softmax warps from the cos/sin
-// table; keys arrive already rotated.
+// table, K rotation in warps 10-11.
 //
 // Exponentials: MUFU ex2.approx.  A compile-time option (JL_X2_POLY_PAIRS)
 // moves some column pairs of each unmasked row to 2^floor(x) * p(x - floor(x))
@@ -62,6 +64,8 @@ constexpr int kStages = 2;
 constexpr int kThreads = 384;  // three warpgroups: softmax 0, softmax 1, producer + MMA
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kRotWarp0 = 10;  // warps 10 and 11 rotate the K tiles
+constexpr int kRotThreads = 64;
 
 constexpr uint32_t kOffQ0 = 0;
 constexpr uint32_t kOffQ1 = kOffQ0 + kTileBytes;
@@ -75,7 +79,8 @@ enum : int {
   kBarKEmpty = kBarKFull + kStages,
   kBarVFull = kBarKEmpty + kStages,
   kBarVEmpty = kBarVFull + kStages,
-  kBarSFull = kBarVEmpty + kStages,  // [2] per head, tcgen05.commit
+  kBarKRot = kBarVEmpty + kStages,   // [kStages] K tile rotated, kRotThreads arrivals
+  kBarSFull = kBarKRot + kStages,    // [2] per head, tcgen05.commit
   // [2][2] per head and part of P, 128 arrivals each; head t's pair at
   // kBarPFull + 4t (the two heads' barriers in different 32-byte sectors)
   kBarPFull = kBarSFull + 2,
@@ -138,6 +143,8 @@ struct KParams {
   int pair_group;  // head pairs whose CTAs are scheduled together (divides Hq / 2)
   int band;   // kBandNone, kBandStd or kBandRem
   int q_off;  // position of query row 0 (a multiple of 128; keys start at 0)
+  int key_mode;  // kKeysRaw or kKeysCached
+  int n_keys;    // keys [0, n_keys) exist (q_off + L)
   float scale_log2;
 };
 
@@ -175,8 +182,7 @@ __device__ __forceinline__ void rotate_q_row(uint8_t *dst, int r, const __nv_bfl
 // chunked prefill); the default prefill runs the instantiation without them.
 template <bool kGeneral>
 __global__ void __launch_bounds__(kThreads, 1)
-    bifocal_prefill_sm100_x2_kernel(const __grid_constant__ CUtensorMap tm_kstd,
-                                    const __grid_constant__ CUtensorMap tm_krem,
+    bifocal_prefill_sm100_x2_kernel(const __grid_constant__ CUtensorMap tm_k,
                                     const __grid_constant__ CUtensorMap tm_v,
                                     const KParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -219,6 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarKEmpty + s), 1);
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarVEmpty + s), 1);
+      mbar_init(bar(kBarKRot + s), kRotThreads);
     }
     mbar_init(bar(kBarDrain), 1);
     *abort_s = 0;
@@ -448,8 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kProducerWarp) {
       // ------------------------------------------------------ TMA producer --
       if (lane == 0) {
-        prefetch_tmap(&tm_kstd);
-        prefetch_tmap(&tm_krem);
+        prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
         PassIter it;
         it.begin(qt + q_off / kBM, p.w, band);
@@ -461,11 +467,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             raise_abort(abort_s, p.status);
             break;
           }
-          const CUtensorMap *km = it.kind() == kStd ? &tm_kstd : &tm_krem;
           mbar_arrive_expect_tx(bar(kBarKFull + s), kTileBytes);
-          tma_load_4d(sb + kOffK + s * kTileBytes, km, bar(kBarKFull + s), 0, hk, kBN * it.j, b);
-          tma_load_4d(sb + kOffK + s * kTileBytes + kHalfBytes, km, bar(kBarKFull + s), 64, hk,
-                      kBN * it.j, b);
+          tma_load_4d(sb + kOffK + s * kTileBytes, &tm_k, bar(kBarKFull + s), 0, hk, kBN * it.j,
+                      b);
+          tma_load_4d(sb + kOffK + s * kTileBytes + kHalfBytes, &tm_k, bar(kBarKFull + s), 64,
+                      hk, kBN * it.j, b);
           ++kiss;
           if (!mbar_wait(bar(kBarVEmpty + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
             raise_abort(abort_s, p.status);
@@ -508,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!wait(kBarQReady + t, qphase[t] & 1)) return false;
             ++qphase[t];
           }
-          if (t == 0 && !wait(kBarKFull + s, (jj / kStages) & 1)) return false;
+          if (t == 0 && !wait(kBarKRot + s, (jj / kStages) & 1)) return false;
           tc_fence_after();
           const uint32_t a0 = sb + (t == 0 ? kOffQ0 : kOffQ1);
           const uint32_t b0 = sb + kOffK + s * kTileBytes;
@@ -565,6 +571,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(bar(kBarDrain), 0);
       }
       __syncwarp();
+    } else {
+      // ------------------------------------------------- K rotation (10-11) --
+      // Each K tile, once the TMA has landed it, is rotated in place to the
+      // positions of its pass and handed to the MMA warp (kBarKRot).  Tile j
+      // of the walk sits in stage j % kStages; the producer refills a stage
+      // only after both score products have read it.
+      const int tid = static_cast<int>(threadIdx.x) - 32 * kRotWarp0;
+      PassIter it;
+      it.begin(qt + q_off / kBM, p.w, band);
+      int n = 0;
+      while (!it.done()) {
+        const int s = n % kStages;
+        if (!mbar_wait(bar(kBarKFull + s), (n / kStages) & 1, abort_s, abort_g, kTimeoutNs)) {
+          raise_abort(abort_s, p.status);
+          break;
+        }
+        rotate_k_tile(smem + kOffK + s * kTileBytes, kBN * it.j, it.kind(), p.key_mode, p.G,
+                      p.n_keys, p.cs, tid, kRotThreads);
+        fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
+        mbar_arrive(bar(kBarKRot + s));
+        ++n;
+        it.next();
+      }
     }
   }
   __syncthreads();
@@ -619,16 +648,12 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  CUtensorMap mks, mkr, mv;
-  const void *krem = a.krem ? a.krem : a.kstd;
-  const void *kstd = a.kstd ? a.kstd : a.krem;
-  // keys [0, q_off + L); the cache-resident tensors (K_std, V) may be longer
-  // per batch entry than that (kv_stride keys)
+  CUtensorMap mk, mv;
+  // keys [0, q_off + L); a cache may be longer per batch entry than that
+  // (kv_stride keys)
   const int keys = a.q_off + a.L;
   const int64_t kvs = a.kv_stride > 0 ? a.kv_stride : keys;
-  if (!make_map(&mks, kstd, a.B, keys, a.Hkv, a.kstd ? kvs : keys) ||
-      !make_map(&mkr, krem, a.B, keys, a.Hkv, a.krem ? keys : kvs) ||
-      !make_map(&mv, a.v, a.B, keys, a.Hkv, kvs))
+  if (!make_map(&mk, a.k, a.B, keys, a.Hkv, kvs) || !make_map(&mv, a.v, a.B, keys, a.Hkv, kvs))
     return cudaErrorInvalidValue;
   KParams p;
   p.q = static_cast<const __nv_bfloat16 *>(a.q);
@@ -644,6 +669,8 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
   p.w = a.w_eff;
   p.band = a.band;
   p.q_off = a.q_off;
+  p.key_mode = a.key_mode;
+  p.n_keys = keys;
   p.n_qtiles = (a.L + kBM - 1) / kBM;
   {
     // whole kv heads per group: kKvPerGroup of them (all when fewer)
@@ -655,9 +682,9 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * (a.Hq / 2);
   if (a.band != 0 || a.q_off != 0)
-    bifocal_prefill_sm100_x2_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mks, mkr, mv, p);
+    bifocal_prefill_sm100_x2_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mv, p);
   else
-    bifocal_prefill_sm100_x2_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mks, mkr, mv, p);
+    bifocal_prefill_sm100_x2_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mv, p);
   return cudaGetLastError();
 }
 

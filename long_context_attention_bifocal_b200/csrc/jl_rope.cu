@@ -1,9 +1,10 @@
-// jl_rope.cu -- the RoPE angle table and the per-call key rotation pass.
+// jl_rope.cu -- the RoPE angle table.
 //
 // RoPE (rotate-half pairs (i, i + D/2), theta_i = base^(-2i/D)) is the position
 // encoding both windows use; the remote window evaluates it at f(x) = floor(x/G)
 // (Jet-Long, bittide paper summary §3.1).  Rotations compose, R(a)R(b) = R(a+b)
-// (techwalker explainer §三), which is what lets every rotation here come from
+// (techwalker explainer §三), which is what lets every rotation of the library
+// (queries and keys in the prefill kernels, the decode's corrections) come from
 // one table of angles p * theta_i.
 #include "jl_internal.h"
 
@@ -30,107 +31,6 @@ __global__ void rope_table_kernel(float2 *__restrict__ cs, int positions, int ha
   }
 }
 
-__device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    x[2 * j] = __uint_as_float(w[j] << 16);
-    x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-  }
-}
-
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// One thread per (key row, 8-pair chunk): reads dims [8c, 8c+8) and
-// [half + 8c, half + 8c + 8) of one key, writes the rotated copies.
-__global__ void rotate_keys_kernel(const __nv_bfloat16 *__restrict__ k,
-                                   __nv_bfloat16 *__restrict__ kstd,
-                                   __nv_bfloat16 *__restrict__ krem,
-                                   const float2 *__restrict__ cs, int64_t rows, int L,
-                                   int Hkv, int D, int G) {
-  const int half = D / 2;
-  const int chunks = half / 8;
-  const int64_t n = rows * chunks;
-  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = idx / chunks;  // (b, l, h) flattened
-    const int c = static_cast<int>(idx - row * chunks);
-    const int l = static_cast<int>((row / Hkv) % L);
-    const int64_t base = row * D + 8 * c;
-    const uint4 u1 = *reinterpret_cast<const uint4 *>(k + base);
-    const uint4 u2 = *reinterpret_cast<const uint4 *>(k + base + half);
-    float x1[8], x2[8];
-    unpack8(u1, x1);
-    unpack8(u2, x2);
-#pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
-      __nv_bfloat16 *dst = pass == 0 ? kstd : krem;
-      if (dst == nullptr) continue;
-      const int p = pass == 0 ? l : l / G;
-      const float2 *t = cs + static_cast<int64_t>(p) * half + 8 * c;
-      float y1[8], y2[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float2 r = __ldg(t + e);
-        y1[e] = x1[e] * r.x - x2[e] * r.y;
-        y2[e] = x1[e] * r.y + x2[e] * r.x;
-      }
-      uint4 o1, o2;
-      o1.x = pack2(y1[0], y1[1]); o1.y = pack2(y1[2], y1[3]);
-      o1.z = pack2(y1[4], y1[5]); o1.w = pack2(y1[6], y1[7]);
-      o2.x = pack2(y2[0], y2[1]); o2.y = pack2(y2[2], y2[3]);
-      o2.z = pack2(y2[4], y2[5]); o2.w = pack2(y2[6], y2[7]);
-      *reinterpret_cast<uint4 *>(dst + base) = o1;
-      *reinterpret_cast<uint4 *>(dst + base + half) = o2;
-    }
-  }
-}
-
-// krem[b, k] = R(f(k) - k) kc[b, k] for keys k < L of a cache rotated at
-// original positions: by -u theta_i with u = k - f(k) >= 0, i.e. with the
-// table row u and the sine negated.  One thread per 8 pairs of one key row.
-__global__ void correct_keys_kernel(const __nv_bfloat16 *__restrict__ kc,
-                                    __nv_bfloat16 *__restrict__ krem,
-                                    const float2 *__restrict__ cs, int64_t rows, int L, int cap,
-                                    int Hkv, int D, int G) {
-  const int half = D / 2;
-  const int chunks = half / 8;
-  const int64_t n = rows * chunks;
-  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = idx / chunks;  // (b, l, h) of the output, flattened
-    const int c = static_cast<int>(idx - row * chunks);
-    const int h = static_cast<int>(row % Hkv);
-    const int l = static_cast<int>((row / Hkv) % L);
-    const int64_t b = row / (static_cast<int64_t>(Hkv) * L);
-    const int64_t src = ((b * cap + l) * Hkv + h) * D + 8 * c;
-    const int64_t dst = row * D + 8 * c;
-    float x1[8], x2[8];
-    unpack8(*reinterpret_cast<const uint4 *>(kc + src), x1);
-    unpack8(*reinterpret_cast<const uint4 *>(kc + src + half), x2);
-    const int u = l - l / G;
-    const float2 *t = cs + static_cast<int64_t>(u) * half + 8 * c;
-    float y1[8], y2[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float2 r = __ldg(t + e);
-      y1[e] = x1[e] * r.x + x2[e] * r.y;
-      y2[e] = x2[e] * r.x - x1[e] * r.y;
-    }
-    uint4 o1, o2;
-    o1.x = pack2(y1[0], y1[1]); o1.y = pack2(y1[2], y1[3]);
-    o1.z = pack2(y1[4], y1[5]); o1.w = pack2(y1[6], y1[7]);
-    o2.x = pack2(y2[0], y2[1]); o2.y = pack2(y2[2], y2[3]);
-    o2.z = pack2(y2[4], y2[5]); o2.w = pack2(y2[6], y2[7]);
-    *reinterpret_cast<uint4 *>(krem + dst) = o1;
-    *reinterpret_cast<uint4 *>(krem + dst + half) = o2;
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_rope_table(float2 *cs, int positions, int D, double base, cudaStream_t s) {
@@ -145,32 +45,4 @@ cudaError_t launch_rope_table(float2 *cs, int positions, int D, double base, cud
   return cudaGetLastError();
 }
 
-cudaError_t launch_rotate_keys(const __nv_bfloat16 *k, __nv_bfloat16 *kstd,
-                               __nv_bfloat16 *krem, RopeTable t, int B, int L,
-                               int Hkv, int D, int G, cudaStream_t s) {
-  const int64_t rows = static_cast<int64_t>(B) * L * Hkv;
-  const int64_t n = rows * (D / 16);
-  const int threads = 256;
-  const int64_t want = (n + threads - 1) / threads;
-  const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
-  const int blocks = static_cast<int>(want < cap ? want : cap);
-  rotate_keys_kernel<<<blocks, threads, 0, s>>>(k, kstd, krem, t.cs, rows, L, Hkv, D, G);
-  return cudaGetLastError();
-}
-
-}  // namespace jl
-
-namespace jl {
-cudaError_t launch_correct_keys(const __nv_bfloat16 *kc, __nv_bfloat16 *krem, RopeTable t,
-                                int B, int L, int cap, int Hkv, int D, int G, cudaStream_t s) {
-  const int64_t rows = static_cast<int64_t>(B) * L * Hkv;
-  const int64_t n = rows * (D / 16);
-  const int threads = 256;
-  const int64_t want = (n + threads - 1) / threads;
-  const int64_t lim = static_cast<int64_t>(sm_count()) * 16;
-  const int blocks = static_cast<int>(want < lim ? want : lim);
-  if (blocks < 1) return cudaSuccess;
-  correct_keys_kernel<<<blocks, threads, 0, s>>>(kc, krem, t.cs, rows, L, cap, Hkv, D, G);
-  return cudaGetLastError();
-}
 }  // namespace jl

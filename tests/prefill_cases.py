@@ -31,7 +31,7 @@ SMALL = [
     (2, 400, 3, 3, 128, 50, 0.5),      # multi-head (group 1), B=2
     (1, 4096, 2, 1, 16, 100, 0.5),     # G = 256: 256 keys share each remapped position
     (1, 1400, 4, 2, 400, 384, 1.0),    # G=4, scale 1.0, window edge on a tile boundary
-    (1, 1300, 2, 1, 350, 451, 1.5),    # G=4, scale 1.5, window edge inside a tile
+    (1, 1300, 2, 1, 350, 451, 1.0),    # G=4, scale 1.0, window edge inside a tile
 ]
 
 

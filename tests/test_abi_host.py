@@ -85,8 +85,6 @@ INVALID, UNSUPPORTED = 1, 2
     (dict(flags=1 << 7), INVALID),
     (dict(flags=1 << 31), INVALID),       # the decode-only test flag
     (dict(dtype=5), INVALID),
-    (dict(ws=FAKE + 16, ws_bytes=1 << 30), INVALID),  # workspace not 256-aligned
-    (dict(ws=FAKE, ws_bytes=10), INVALID),            # workspace too small
 ])
 def test_prefill_rejects(lib, kw, code):
     assert _prefill(lib, **kw) == code
@@ -122,8 +120,10 @@ def test_decode_rejects(lib, kw, code):
 
 
 def test_workspace_sizes(lib):
-    assert lib.jl_bifocal_prefill_workspace_size(1, 131072, 8, 128, 0) == 2 * 131072 * 8 * 128 * 2
+    # keys are rotated inside the prefill kernels: no workspace at any size
+    assert lib.jl_bifocal_prefill_workspace_size(1, 131072, 8, 128, 0) == 0
     assert lib.jl_bifocal_prefill_workspace_size(1, 100, 8, 64, 1) == 0
+    assert lib.jl_bifocal_prefill_chunk_workspace_size(1, 131072 - 16384, 16384, 8, 128) == 0
     n = lib.jl_bifocal_decode_workspace_size(1, 32, 8, 128, 131071)
     assert n > 0 and n % 4 == 0
     assert lib.jl_bifocal_decode_workspace_size(1, 32, 8, 128, -1) == 0
@@ -166,8 +166,8 @@ def test_prefill_3pass_workspace_size(lib):
     B, L, Hq, Hkv, D = 1, 1000, 4, 2, 128
     n = lib.jl_bifocal_prefill_3pass_workspace_size(B, L, Hq, Hkv, D)
     up = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    keys = 2 * up(B * L * Hkv * D * 2)
-    assert n == keys + 2 * up(B * L * Hq * D * 2) + 2 * up(B * Hq * L * 4)
+    # O_B and O_C (bf16) and their lse; the keys are rotated inside the kernels
+    assert n == 2 * up(B * L * Hq * D * 2) + 2 * up(B * Hq * L * 4)
 
 
 def _decode_batched(lib, pos=(100, 5), **kw):
@@ -222,8 +222,6 @@ def _prefill_chunk(lib, **kw):
     (dict(cap=500), INVALID),                # q_offset + Lq > cap
     (dict(D=64), UNSUPPORTED),
     (dict(Lq=0), INVALID),
-    (dict(ws=FAKE, ws_bytes=10), INVALID),
-    (dict(ws=FAKE + 16, ws_bytes=1 << 30), INVALID),
     (dict(flags=1 << 31), INVALID),
 ])
 def test_prefill_chunk_rejects(lib, kw, code):

@@ -105,14 +105,19 @@ def test_bf16_bifocal_differs_from_plain_when_g_gt_1(jl):
     assert (a[0].float() - b[0].float()).abs().max().item() > 1e-2
 
 
-def test_explicit_workspace_matches_library_scratch(jl):
+def test_needs_no_workspace_and_repeats_bitwise(jl):
+    """The keys are rotated inside the kernel: the call needs no workspace, and
+    a workspace handed to it is neither needed nor written; repeated calls give
+    identical bits."""
+    assert jl.prefill_workspace_size(1, 900, 2, 128) == 0
     q, k, v = W.prefill_inputs(1, 900, 4, 2, 128, seed=9)
     kw = dict(w_local=128, w_pretrained=300, rope_base=1e6)
     a = run_prefill(jl, q, k, v, **kw)
-    ws = torch.empty(jl.prefill_workspace_size(1, 900, 2, 128), dtype=torch.uint8, device=DEV)
+    ws = torch.full((4096,), 7, dtype=torch.uint8, device=DEV)
     b = jl.bifocal_prefill(q.to(DEV), k.to(DEV), v.to(DEV), workspace=ws, **kw)
     jl.check_device_status()
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    assert bool((ws == 7).all())
 
 
 # ---------------------------------- full sizes, sampled rows per head ----
