@@ -132,53 +132,206 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8]) {
 // explainer §三: rotations compose, R(a) R(b) = R(a + b)).
 enum : int { kKeysRaw = 0, kKeysCached = 1 };
 
-// Rotates a 128-key tile in shared memory, in place, for a pass of class
-// `kind` (kStd / kRem) over keys k0 .. k0 + 127, bf16 in the 128-byte-swizzled
-// K-major layout the TMA wrote: dims 0-63 in the first 16 KB half, 64-127 in
-// the second, pair (i, i + 64) at the same offset of the two halves.  The
-// `nthr` threads calling it (thread index `tid`) split the 128 x 8 chunks of
-// eight pairs between them; a thread's lanes of one warp take four rows of
-// eight chunks, so table reads and shared-memory accesses stay contiguous.
-// Rows at or past n_keys (zero fill beyond the sequence) are left alone.
-// Arithmetic: fp32 with the fp32 table value of (cos, sin)(p theta_i), one
-// rounding to bf16 at the end.
-__device__ __forceinline__ void rotate_k_tile(uint8_t *tile, int k0, int kind, int key_mode,
-                                              int G, int n_keys, const float2 *cs, int tid,
-                                              int nthr) {
-  if (key_mode == kKeysCached && kind == kStd) return;  // already at original positions
-#pragma unroll 1
-  for (int item = tid; item < kBN * 8; item += nthr) {
-    const int r = item >> 3, c = item & 7;
-    const int k = k0 + r;
-    if (k >= n_keys) continue;
-    int p;
-    float sgn = 1.f;
-    if (key_mode == kKeysRaw) {
-      p = kind == kStd ? k : k / G;
-    } else {
-      p = k - k / G;  // R(f(k) - k) = R(-u): the table row u with the sine negated
-      sgn = -1.f;
-    }
-    uint4 *a1 = reinterpret_cast<uint4 *>(tile + swz(r, c));
-    uint4 *a2 = reinterpret_cast<uint4 *>(tile + kHalfBytes + swz(r, c));
-    float x1[8], x2[8];
-    unpack8(*a1, x1);
-    unpack8(*a2, x2);
-    const float4 *t = reinterpret_cast<const float4 *>(cs + static_cast<int64_t>(p) * 64 + 8 * c);
-    uint32_t lo[4], hi[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float4 r2 = __ldg(t + e);  // (cos, sin) of pairs 2e and 2e + 1
-      const float s0 = sgn * r2.y, s1 = sgn * r2.w;
-      lo[e] = pack_bf16x2(x1[2 * e] * r2.x - x2[2 * e] * s0,
-                          x1[2 * e + 1] * r2.z - x2[2 * e + 1] * s1);
-      hi[e] = pack_bf16x2(x1[2 * e] * s0 + x2[2 * e] * r2.x,
-                          x1[2 * e + 1] * s1 + x2[2 * e + 1] * r2.z);
-    }
-    *a1 = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    *a2 = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+// In-place rotation of part of a 128-key tile in shared memory (bf16, the
+// 128-byte-swizzled K-major layout the TMA wrote: dims 0-63 in the first
+// 16 KB half, 64-127 in the second, so pair (i, i + 64) sits at the same
+// offset of the two halves) to the positions of a pass.
+//
+// One thread's slice: the eight pairs 8c .. 8c + 7 (one 16-byte chunk of each
+// half) of four consecutive keys kl .. kl + 3 of the tile.  Their positions p
+// advance by 0 or 1 per key (k, floor(k / G), or k - floor(k / G) for a cache
+// at original positions), so the table is read once, at the first key, and
+// the factors then move on by R(p + 1) = R(p) R(1) (a complex multiplication
+// with row 1 of the table, kept in shared memory as `step`) where p advances.
+// All four keys' words are loaded before any is rotated, so one shared-memory
+// latency covers the slice.  Arithmetic in fp32, one rounding to bf16.
+struct KeySlice {
+  int c;   // chunk of pairs
+  int kl;  // first key of the slice within the tile
+
+  // position of key k in a pass of class `kind`; -1 when the keys are used as
+  // they are (cached keys in a local pass)
+  static __device__ __forceinline__ int position(int k, int kind, int key_mode, int G) {
+    if (key_mode == kKeysRaw) return kind == kStd ? k : k / G;
+    return kind == kStd ? -1 : k - k / G;
   }
-}
+
+  // pulls the slice's table entries into L1 ahead of rotate()
+  __device__ void prefetch(const float2 *cs, int k0, int kind, int key_mode, int G,
+                           int n_keys) const {
+    const int k = k0 + kl;
+    if (k >= n_keys) return;
+    const int p = position(k, kind, key_mode, G);
+    if (p < 0) return;
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(cs + static_cast<int64_t>(p) * 64 + 8 * c));
+  }
+
+  __device__ void rotate(uint8_t *tile, const float2 *cs, const float2 *step, int k0, int kind,
+                         int key_mode, int G, int n_keys) const {
+    const int k = k0 + kl;
+    const int rows = min(4, n_keys - k);
+    if (rows <= 0) return;
+    const int p = position(k, kind, key_mode, G);
+    if (p < 0) return;
+    const bool cached = key_mode == kKeysCached;
+    const bool every = key_mode == kKeysRaw && kind == kStd;  // p = k: a step per key
+    const float sg = cached ? -1.f : 1.f;  // R(-u) for the cached keys' correction
+    uint4 w1[4], w2[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (u < rows) {
+        const uint32_t off = swz(kl + u, c);
+        w1[u] = *reinterpret_cast<const uint4 *>(tile + off);
+        w2[u] = *reinterpret_cast<const uint4 *>(tile + kHalfBytes + off);
+      }
+    }
+    float cf[8], sf[8];
+    {
+      const float4 *t = reinterpret_cast<const float4 *>(cs + static_cast<int64_t>(p) * 64 + 8 * c);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float4 v = __ldg(t + e);
+        cf[2 * e] = v.x;
+        sf[2 * e] = sg * v.y;
+        cf[2 * e + 1] = v.z;
+        sf[2 * e + 1] = sg * v.w;
+      }
+    }
+    int m = k % G;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (u < rows) {
+        const uint32_t a1[4] = {w1[u].x, w1[u].y, w1[u].z, w1[u].w};
+        const uint32_t a2[4] = {w2[u].x, w2[u].y, w2[u].z, w2[u].w};
+        uint32_t o1[4], o2[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float x1a = __uint_as_float(a1[q] << 16), x1b = __uint_as_float(a1[q] & 0xFFFF0000u);
+          const float x2a = __uint_as_float(a2[q] << 16), x2b = __uint_as_float(a2[q] & 0xFFFF0000u);
+          const int e = 2 * q;
+          o1[q] = sm100::pack_bf16x2(fmaf(x1a, cf[e], -x2a * sf[e]),
+                                     fmaf(x1b, cf[e + 1], -x2b * sf[e + 1]));
+          o2[q] = sm100::pack_bf16x2(fmaf(x1a, sf[e], x2a * cf[e]),
+                                     fmaf(x1b, sf[e + 1], x2b * cf[e + 1]));
+        }
+        const uint32_t off = swz(kl + u, c);
+        *reinterpret_cast<uint4 *>(tile + off) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+        *reinterpret_cast<uint4 *>(tile + kHalfBytes + off) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+        // next key: k mod G, and whether its position moves on (f grows at
+        // multiples of G; u = k - f everywhere else)
+        m = (m + 1 == G) ? 0 : m + 1;
+        if (u + 1 < rows && (every || (cached ? (m != 0) : (m == 0)))) {
+          const float4 *st4 = reinterpret_cast<const float4 *>(step + 8 * c);
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float4 v = st4[e2];  // (cos, sin)(theta) of pairs 2 e2, 2 e2 + 1
+            const float c1[2] = {v.x, v.z}, s1[2] = {sg * v.y, sg * v.w};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int e = 2 * e2 + h;
+              const float cn = fmaf(cf[e], c1[h], -sf[e] * s1[h]);
+              sf[e] = fmaf(cf[e], s1[h], sf[e] * c1[h]);
+              cf[e] = cn;
+            }
+          }
+        }
+      }
+    }
+  }
+};
+
+// The same rotation by NTHR dedicated threads (a multiple of 16) over a whole
+// tile: thread t owns four pairs i0 .. i0 + 3 (i0 = 4 * (t % 16)), one 8-byte
+// word of each half, of kRows = 128 * 16 / NTHR consecutive keys, moving its
+// factors on by the step table as KeySlice does and loading the next key's
+// words before rotating the current one.
+template <int NTHR>
+struct KeyRotator {
+  static constexpr int kRows = kBN * 16 / NTHR;
+  const float4 *step;  // (cos, sin)(theta_i) of the thread's pairs, two per float4
+  int i0;              // first pair of this thread
+  int kb;              // first key of the thread's block within a tile
+
+  __device__ void init(const float2 *step_smem, int tid) {
+    i0 = 4 * (tid & 15);
+    kb = kRows * (tid >> 4);
+    step = reinterpret_cast<const float4 *>(step_smem + i0);
+  }
+
+  struct Start {
+    float4 a, b;
+    int m;      // k mod G of the first key
+    int rows;   // keys of the block to rotate (0: none)
+  };
+  // the block's first position and its table entries, read ahead of the wait
+  // for the tile
+  __device__ Start start(const float2 *cs, int k0, int kind, int key_mode, int G,
+                         int n_keys) const {
+    Start st;
+    const int k = k0 + kb;
+    const int p = k < n_keys ? KeySlice::position(k, kind, key_mode, G) : -1;
+    st.rows = p < 0 ? 0 : min(kRows, n_keys - k);
+    st.m = k % G;
+    const float4 *t =
+        reinterpret_cast<const float4 *>(cs + static_cast<int64_t>(p < 0 ? 0 : p) * 64 + i0);
+    st.a = __ldg(t);
+    st.b = __ldg(t + 1);
+    return st;
+  }
+
+  __device__ void rotate(uint8_t *tile, const Start &st, int kind, int key_mode, int G) const {
+    if (st.rows <= 0) return;
+    const bool cached = key_mode == kKeysCached;
+    const bool every = key_mode == kKeysRaw && kind == kStd;
+    const float sg = cached ? -1.f : 1.f;
+    float c[4] = {st.a.x, st.a.z, st.b.x, st.b.z};
+    float s[4] = {sg * st.a.y, sg * st.a.w, sg * st.b.y, sg * st.b.w};
+    const int c_off = i0 >> 3, h_off = (i0 & 4) * 2;  // 16-byte chunk, 8-byte half
+    int m = st.m;
+    uint32_t off = swz(kb, c_off) + h_off;
+    uint2 w1 = *reinterpret_cast<const uint2 *>(tile + off);
+    uint2 w2 = *reinterpret_cast<const uint2 *>(tile + kHalfBytes + off);
+#pragma unroll 1
+    for (int n = 0; n < st.rows; ++n) {
+      const uint32_t noff = swz(kb + n + 1, c_off) + h_off;
+      uint2 n1 = w1, n2 = w2;
+      if (n + 1 < st.rows) {
+        n1 = *reinterpret_cast<const uint2 *>(tile + noff);
+        n2 = *reinterpret_cast<const uint2 *>(tile + kHalfBytes + noff);
+      }
+      const float x1[4] = {__uint_as_float(w1.x << 16), __uint_as_float(w1.x & 0xFFFF0000u),
+                           __uint_as_float(w1.y << 16), __uint_as_float(w1.y & 0xFFFF0000u)};
+      const float x2[4] = {__uint_as_float(w2.x << 16), __uint_as_float(w2.x & 0xFFFF0000u),
+                           __uint_as_float(w2.y << 16), __uint_as_float(w2.y & 0xFFFF0000u)};
+      float y1[4], y2[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        y1[e] = fmaf(x1[e], c[e], -x2[e] * s[e]);
+        y2[e] = fmaf(x1[e], s[e], x2[e] * c[e]);
+      }
+      *reinterpret_cast<uint2 *>(tile + off) =
+          make_uint2(sm100::pack_bf16x2(y1[0], y1[1]), sm100::pack_bf16x2(y1[2], y1[3]));
+      *reinterpret_cast<uint2 *>(tile + kHalfBytes + off) =
+          make_uint2(sm100::pack_bf16x2(y2[0], y2[1]), sm100::pack_bf16x2(y2[2], y2[3]));
+      m = (m + 1 == G) ? 0 : m + 1;
+      if (every || (cached ? (m != 0) : (m == 0))) {
+        const float4 t01 = step[0], t23 = step[1];
+        const float c1[4] = {t01.x, t01.z, t23.x, t23.z};
+        const float s1[4] = {t01.y, t01.w, t23.y, t23.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float sd = sg * s1[e];
+          const float cn = fmaf(c[e], c1[e], -s[e] * sd);
+          s[e] = fmaf(c[e], sd, s[e] * c1[e]);
+          c[e] = cn;
+        }
+      }
+      off = noff;
+      w1 = n1;
+      w2 = n2;
+    }
+  }
+};
 
 // 2^x on the FMA/ALU pipes instead of the MUFU unit, for x <= 8:
 // 2^floor(x) * p(x - floor(x)) with a cubic p fitted by weighted least squares

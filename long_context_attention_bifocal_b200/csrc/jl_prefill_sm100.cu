@@ -33,9 +33,15 @@
 //   warp 5     allocates TMEM and issues every tcgen05.mma from one thread:
 //              S = Q K^T (M=N=128, K=128: 8 x K16 steps) into one of two TMEM
 //              S buffers, and O += P V into the TMEM O accumulator.
-//   warps 6-7  rotate each K tile in shared memory, in place, to the pass's
+//   warps 6-7  idle (they complete the second warpgroup)
+//   warps 8-11 rotate each K tile in shared memory, in place, to the pass's
 //              positions (R(k) or R(f(k)) from the cos/sin table) before the
-//              score product reads it: RoPE applied on the fly.
+//              score product reads it: RoPE applied on the fly.  Four warps,
+//              one per SM sub-partition.
+// Registers: launched at 168 a thread (sm_100 allocates them per four warps);
+// the producer/MMA warpgroup gives 96 back per thread and the softmax
+// warpgroup takes 48 of them, so a softmax thread holds its whole S row
+// (128 x 216 + 128 x 72 + 128 x 168 <= 384 x 168).
 // Every mbarrier wait is bounded (1 s); a thread that gives up raises the
 // CTA's abort flag and the device status word, after which all CTAs drain and
 // return without touching their outputs further.
@@ -55,9 +61,9 @@ using namespace prefill;
 
 // shared-memory layout (bytes from the 1 KiB-aligned base), barriers, TMEM
 constexpr int kStages = 3;
-constexpr int kThreads = 256;
-constexpr int kRotWarp0 = 6;  // warps 6 and 7 rotate the K tiles
-constexpr int kRotThreads = 64;
+constexpr int kThreads = 384;
+constexpr int kRotWarp0 = 8;  // warps 8-11 rotate the K tiles
+constexpr int kRotThreads = 128;
 
 constexpr uint32_t kOffQ = 0;  // the Q variant of the current phase
 constexpr uint32_t kOffK = kOffQ + kTileBytes;
@@ -82,7 +88,8 @@ enum : int {
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
 constexpr uint32_t kOffSkip = kOffAbort + 4;
-constexpr uint32_t kSmemUsed = kOffSkip + 4;
+constexpr uint32_t kOffStep = (kOffSkip + 4 + 15) & ~15u;  // 64 x float2: R(1) per pair
+constexpr uint32_t kSmemUsed = kOffStep + 64 * 8;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // room to align the base to 1 KiB
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
@@ -170,6 +177,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(sb + kOffTmemSlot, kTmemCols);
     tmem_relinquish();
   }
+  // the key rotation's step factors: table row 1, (cos, sin)(theta_i)
+  if (threadIdx.x < 64)
+    reinterpret_cast<float2 *>(smem + kOffStep)[threadIdx.x] = p.cs[64 + threadIdx.x];
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + kOffTmemSlot);
@@ -177,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (!skip) {
     if (warp < 4) {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
       // ------------------------------------------------ softmax warpgroup --
       const int r = threadIdx.x;  // query row within the tile == TMEM lane
       const int row_i = kBM * qt + r;    // row of the q / out / lse tensors
@@ -384,7 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.lse[(static_cast<int64_t>(b) * p.Hq + hq) * p.L + row_i] =
               (m + __log2f(l)) * 0.69314718055994530942f;
       }
-    } else if (warp == 4) {
+    } else if (warp < kRotWarp0) {
+     asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+     if (warp == 4) {
       // ------------------------------------------------------ TMA producer --
       if (lane == 0) {
         prefetch_tmap(&tm_k);
@@ -495,24 +508,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(bar(kBarDrain), 0);
       }
       __syncwarp();
+     }
     } else {
-      // --------------------------------------------------- K rotation (6-7) --
+      // -------------------------------------------------- K rotation (8-11) --
       // Pass n's K tile sits in stage n % kStages; once the TMA has landed it,
       // it is rotated in place to its pass's positions and handed to the MMA
       // warp (kBarKRot).  The producer refills a stage only after the score
       // product has read it.
-      const int tid = static_cast<int>(threadIdx.x) - 32 * kRotWarp0;
+      KeyRotator<kRotThreads> rot;
+      rot.init(reinterpret_cast<const float2 *>(smem + kOffStep),
+               static_cast<int>(threadIdx.x) - 32 * kRotWarp0);
       PassIter t;
       t.begin(qt + q_off / kBM, p.w, band);
       int n = 0;
       while (!t.done()) {
         const int s = n % kStages;
+        const int k0 = kBN * t.j, kind = t.kind();
+        // the table read for this tile goes out before the wait for its keys
+        const auto st = rot.start(p.cs, k0, kind, p.key_mode, p.G, p.n_keys);
         if (!mbar_wait(bar(kBarKFull + s), (n / kStages) & 1, abort_s, abort_g, kTimeoutNs)) {
           raise_abort(abort_s, p.status);
           break;
         }
-        rotate_k_tile(smem + kOffK + s * kTileBytes, kBN * t.j, t.kind(), p.key_mode, p.G,
-                      p.n_keys, p.cs, tid, kRotThreads);
+        rot.rotate(smem + kOffK + s * kTileBytes, st, kind, p.key_mode, p.G);
         fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
         mbar_arrive(bar(kBarKRot + s));
         ++n;

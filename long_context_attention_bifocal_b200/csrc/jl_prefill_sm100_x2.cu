@@ -12,15 +12,20 @@
 // Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax of head 0: thread r = query row r = TMEM lane r of S0/O0
 //   warps 4-7  softmax of head 1: the same on S1/O1
-//   warp 8     TMA producer: raw K tile and V tile into a 2-stage ring
+//              Between passes, while its next S is being computed, each
+//              softmax thread also rotates its slice (4 keys x 8 pairs) of the
+//              K tile two passes ahead in shared memory, in place, to that
+//              pass's positions (R(k) or R(f(k)) from the cos/sin table): RoPE
+//              applied on the fly, with no rotated copy of the keys in global
+//              memory.  Head 0's warps take keys 0-63, head 1's keys 64-127.
+//   warp 8     TMA producer of the raw K tiles (3-stage ring)
 //   warp 9     TMEM allocation and every tcgen05.mma, from one thread
-//   warps 10-11 rotate each K tile in shared memory, in place, to the pass's
-//              positions (R(k) or R(f(k)) from the cos/sin table) before the
-//              score product reads it: RoPE applied on the fly, with no
-//              rotated copy of the keys in global memory
+//   warp 10    TMA producer of the V tiles (2-stage ring)
+//   warp 11    idle (it completes the third warpgroup)
 // Registers: launched at 168 a thread; the third warpgroup drops to 72 and the
-// softmax warpgroups rise to 216 (setmaxnreg), so a softmax thread holds its
-// whole S row and reads S from TMEM once per pass.
+// softmax warpgroups rise to 216 (setmaxnreg: 2 x 128 x 216 + 128 x 72 =
+// 384 x 168), so a softmax thread holds its whole S row and reads S from TMEM
+// once per pass.
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.  After the
 // softmax has read S_t into registers it writes P_t (bf16, two per column) into
 // the first 64 columns of S_t, and O_t += P_t V takes P_t straight from TMEM,
@@ -34,7 +39,7 @@
 // tile all come before its local passes, so Q_rem is used first and is then
 // overwritten in place by Q_std (one switch per tile, signalled through the
 // q_ready barrier).  Q rotation runs in the softmax warps from the cos/sin
-// table, K rotation in warps 10-11.
+// table, K rotation in the softmax warps between passes.
 //
 // Exponentials: MUFU ex2.approx.  A compile-time option (JL_X2_POLY_PAIRS)
 // moves some column pairs of each unmasked row to 2^floor(x) * p(x - floor(x))
@@ -60,27 +65,31 @@ namespace {
 using namespace sm100;
 using namespace prefill;
 
-constexpr int kStages = 2;
-constexpr int kThreads = 384;  // three warpgroups: softmax 0, softmax 1, producer + MMA
-constexpr int kProducerWarp = 8;
+constexpr int kKStages = 3;  // K ring: a tile is loaded, then rotated, then read by S
+constexpr int kVStages = 2;
+constexpr int kThreads = 384;  // softmax 0, softmax 1, producers + MMA
+constexpr int kProducerWarp = 8;   // K tiles
+constexpr int kVProducerWarp = 10;  // V tiles
 constexpr int kMmaWarp = 9;
-constexpr int kRotWarp0 = 10;  // warps 10 and 11 rotate the K tiles
-constexpr int kRotThreads = 64;
+constexpr int kRotThreads = 256;  // the softmax threads rotate the K tiles
+// register budgets after setmaxnreg (2 x 216 + 72 = 3 x 168)
+constexpr int kRegsSoftmax = 216;
+constexpr int kRegsWg2 = 72;
 
 constexpr uint32_t kOffQ0 = 0;
 constexpr uint32_t kOffQ1 = kOffQ0 + kTileBytes;
 constexpr uint32_t kOffK = kOffQ1 + kTileBytes;
-constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
-constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + kVStages * kTileBytes;
 
 enum : int {
   kBarQReady = 0,                  // [2] per head, 128 arrivals
-  kBarKFull = kBarQReady + 2,      // [kStages]
-  kBarKEmpty = kBarKFull + kStages,
-  kBarVFull = kBarKEmpty + kStages,
-  kBarVEmpty = kBarVFull + kStages,
-  kBarKRot = kBarVEmpty + kStages,   // [kStages] K tile rotated, kRotThreads arrivals
-  kBarSFull = kBarKRot + kStages,    // [2] per head, tcgen05.commit
+  kBarKFull = kBarQReady + 2,      // [kKStages]
+  kBarKEmpty = kBarKFull + kKStages,
+  kBarKRot = kBarKEmpty + kKStages,  // [kKStages] K tile rotated, one arrival per softmax thread
+  kBarVFull = kBarKRot + kKStages,   // [kVStages]
+  kBarVEmpty = kBarVFull + kVStages,
+  kBarSFull = kBarVEmpty + kVStages, // [2] per head, tcgen05.commit
   // [2][2] per head and part of P, 128 arrivals each; head t's pair at
   // kBarPFull + 4t (the two heads' barriers in different 32-byte sectors)
   kBarPFull = kBarSFull + 2,
@@ -92,7 +101,8 @@ enum : int {
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
 constexpr uint32_t kOffSkip = kOffAbort + 4;
-constexpr uint32_t kSmemUsed = kOffSkip + 4;
+constexpr uint32_t kOffStep = (kOffSkip + 4 + 15) & ~15u;  // 64 x float2: R(1) per pair
+constexpr uint32_t kSmemUsed = kOffStep + 64 * 8;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
@@ -220,12 +230,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 2; ++c) mbar_init(bar(kBarPFull + 4 * t + c), 128);
       mbar_init(bar(kBarODone + t), 1);
     }
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarKEmpty + s), 1);
+      mbar_init(bar(kBarKRot + s), kRotThreads);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarVEmpty + s), 1);
-      mbar_init(bar(kBarKRot + s), kRotThreads);
     }
     mbar_init(bar(kBarDrain), 1);
     *abort_s = 0;
@@ -236,6 +248,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(sb + kOffTmemSlot, kTmemCols);
     tmem_relinquish();
   }
+  // the key rotation's step factors: table row 1, (cos, sin)(theta_i)
+  if (threadIdx.x < 64)
+    reinterpret_cast<float2 *>(smem + kOffStep)[threadIdx.x] = p.cs[64 + threadIdx.x];
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + kOffTmemSlot);
@@ -243,13 +258,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (!skip) {
     // Registers are launched at 168 a thread; the producer/MMA warpgroup gives
-    // 128 back per thread so that each softmax thread may hold a whole S row
-    // (2 x 128 x 216 + 128 x 72 = 384 x 168).
-    if (warp < 8)
-      asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
-    else
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+    // 96 back per thread so that each softmax thread may hold a whole S row
+    // (2 x 128 x 216 + 128 x 72 = 384 x 168).  Each warpgroup changes its
+    // budget inside its own branch, so that the compiler allocates each role's
+    // code within that role's budget.
     if (warp < 8) {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
       // --------------------------------------------- softmax warpgroups --
       const int t = warp >> 2;           // head of this warpgroup
       const int r = threadIdx.x & 127;   // query row == TMEM lane
@@ -273,10 +287,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(bar(kBarQReady + t));
 
+      // K rotation: this thread's slice of every K tile of the walk, tile n
+      // (stage n % kKStages) two passes ahead of the softmax
+      KeySlice ks;
+      ks.c = r & 7;
+      ks.kl = 64 * t + 4 * (r >> 3);
+      const float2 *step = reinterpret_cast<const float2 *>(smem + kOffStep);
+      PassIter rit;
+      rit.begin(qt + q_off / kBM, p.w, band);
+      int rot_n = 0;
+      auto rotate_next = [&]() -> bool {
+        if (rit.done()) return true;
+        const int s = rot_n % kKStages;
+        // uniform across the warp, like every wait of the softmax warps
+        if (!warp_wait(bar(kBarKFull + s), (rot_n / kKStages) & 1, abort_s, abort_g))
+          return false;
+        ks.rotate(smem + kOffK + s * kTileBytes, p.cs, step, kBN * rit.j, rit.kind(), p.key_mode,
+                  p.G, p.n_keys);
+        fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
+        mbar_arrive(bar(kBarKRot + s));
+        ++rot_n;
+        rit.next();
+        return true;
+      };
+      bool ok = rotate_next() && rotate_next();
+
       float m = -INFINITY, l = 0.f;
       int j = 0;
-      bool ok = true;
-      while (!it.done()) {
+      while (ok && !it.done()) {
+        if (!rit.done())  // the next slice's table entries, into L1 during the wait
+          ks.prefetch(p.cs, kBN * rit.j, rit.kind(), p.key_mode, p.G, p.n_keys);
         if (!warp_wait(bar(kBarSFull + t), j & 1, abort_s, abort_g)) {
           ok = false;
           break;
@@ -422,6 +462,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l = l * alpha + rs;
         ++j;
+        // the tile two passes ahead, while this head's next S is computed
+        if (!rotate_next()) {
+          ok = false;
+          break;
+        }
       }
       ok = __all_sync(0xffffffffu, ok);
       if (ok && !warp_wait(bar(kBarODone + t), (j - 1) & 1, abort_s, abort_g)) ok = false;
@@ -452,43 +497,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.lse[(static_cast<int64_t>(b) * p.Hq + hq) * p.L + row_i] =
               (m + __log2f(l)) * 0.69314718055994530942f;
       }
-    } else if (warp == kProducerWarp) {
-      // ------------------------------------------------------ TMA producer --
+    } else {
+     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsWg2));
+     if (warp == kProducerWarp || warp == kVProducerWarp) {
+      // ------------------------------------------- TMA producers (K and V) --
+      // Warp 8 loads the raw K tiles of the walk into a kKStages ring, warp 10
+      // the V tiles into a kVStages ring; pass n's tiles sit in stage
+      // n % stages of each.
       if (lane == 0) {
-        prefetch_tmap(&tm_k);
-        prefetch_tmap(&tm_v);
+        const bool is_k = warp == kProducerWarp;
+        const CUtensorMap *map = is_k ? &tm_k : &tm_v;
+        const int stages = is_k ? kKStages : kVStages;
+        const uint32_t base = sb + (is_k ? kOffK : kOffV);
+        const int full = is_k ? kBarKFull : kBarVFull, empty = is_k ? kBarKEmpty : kBarVEmpty;
+        prefetch_tmap(map);
         PassIter it;
         it.begin(qt + q_off / kBM, p.w, band);
-        int kiss = 0, viss = 0;
+        int n = 0;
         while (!it.done()) {
-          const int s = kiss % kStages;
-          const uint32_t ph = (kiss / kStages) & 1;
-          if (!mbar_wait(bar(kBarKEmpty + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
+          const int s = n % stages;
+          if (!mbar_wait(bar(empty + s), ((n / stages) & 1) ^ 1u, abort_s, abort_g, kTimeoutNs)) {
             raise_abort(abort_s, p.status);
             break;
           }
-          mbar_arrive_expect_tx(bar(kBarKFull + s), kTileBytes);
-          tma_load_4d(sb + kOffK + s * kTileBytes, &tm_k, bar(kBarKFull + s), 0, hk, kBN * it.j,
+          mbar_arrive_expect_tx(bar(full + s), kTileBytes);
+          tma_load_4d(base + s * kTileBytes, map, bar(full + s), 0, hk, kBN * it.j, b);
+          tma_load_4d(base + s * kTileBytes + kHalfBytes, map, bar(full + s), 64, hk, kBN * it.j,
                       b);
-          tma_load_4d(sb + kOffK + s * kTileBytes + kHalfBytes, &tm_k, bar(kBarKFull + s), 64,
-                      hk, kBN * it.j, b);
-          ++kiss;
-          if (!mbar_wait(bar(kBarVEmpty + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
-            raise_abort(abort_s, p.status);
-            break;
-          }
-          mbar_arrive_expect_tx(bar(kBarVFull + s), kTileBytes);
-          tma_load_4d(sb + kOffV + s * kTileBytes, &tm_v, bar(kBarVFull + s), 0, hk, kBN * it.j,
-                      b);
-          tma_load_4d(sb + kOffV + s * kTileBytes + kHalfBytes, &tm_v, bar(kBarVFull + s), 64,
-                      hk, kBN * it.j, b);
-          ++viss;
+          ++n;
           it.next();
         }
-        for (int d = (kiss > kStages ? kiss - kStages : 0); d < kiss; ++d)
-          drain_wait(bar(kBarKFull + d % kStages), (d / kStages) & 1);
-        for (int d = (viss > kStages ? viss - kStages : 0); d < viss; ++d)
-          drain_wait(bar(kBarVFull + d % kStages), (d / kStages) & 1);
+        // never leave with a copy in flight into this CTA's shared memory
+        for (int d = (n > stages ? n - stages : 0); d < n; ++d)
+          drain_wait(bar(full + d % stages), (d / stages) & 1);
       }
       __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -509,16 +550,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         int qphase[2] = {0, 0};
         auto issue_s = [&](int t, int jj, int kind_changed) -> bool {
-          const int s = jj % kStages;
+          const int s = jj % kKStages;
           if (kind_changed) {
             if (!wait(kBarQReady + t, qphase[t] & 1)) return false;
             ++qphase[t];
           }
-          if (t == 0 && !wait(kBarKRot + s, (jj / kStages) & 1)) return false;
+          if (t == 0 && !wait(kBarKRot + s, (jj / kKStages) & 1)) return false;
           tc_fence_after();
           const uint32_t a0 = sb + (t == 0 ? kOffQ0 : kOffQ1);
           const uint32_t b0 = sb + kOffK + s * kTileBytes;
-#pragma unroll
+          // a rolled loop: its eight issues take a few tens of cycles against
+          // the product's 512, and it keeps no descriptor live across steps
+#pragma unroll 1
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
             umma_bf16(tmem + tm_s(t), sdesc_sw128(a0 + off, 16, 1024),
@@ -529,8 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         auto issue_pv = [&](int t, int jj) -> bool {
-          const int s = jj % kStages;
-          if (t == 0 && !wait(kBarVFull + s, (jj / kStages) & 1)) return false;
+          const int s = jj % kVStages;
+          if (t == 0 && !wait(kBarVFull + s, (jj / kVStages) & 1)) return false;
           const uint32_t vb = sb + kOffV + s * kTileBytes;
           // P_t arrives in two parts; each is multiplied as soon as it is
           // released.  Each part's steps are a loop with compile-time bounds
@@ -571,29 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(bar(kBarDrain), 0);
       }
       __syncwarp();
-    } else {
-      // ------------------------------------------------- K rotation (10-11) --
-      // Each K tile, once the TMA has landed it, is rotated in place to the
-      // positions of its pass and handed to the MMA warp (kBarKRot).  Tile j
-      // of the walk sits in stage j % kStages; the producer refills a stage
-      // only after both score products have read it.
-      const int tid = static_cast<int>(threadIdx.x) - 32 * kRotWarp0;
-      PassIter it;
-      it.begin(qt + q_off / kBM, p.w, band);
-      int n = 0;
-      while (!it.done()) {
-        const int s = n % kStages;
-        if (!mbar_wait(bar(kBarKFull + s), (n / kStages) & 1, abort_s, abort_g, kTimeoutNs)) {
-          raise_abort(abort_s, p.status);
-          break;
-        }
-        rotate_k_tile(smem + kOffK + s * kTileBytes, kBN * it.j, it.kind(), p.key_mode, p.G,
-                      p.n_keys, p.cs, tid, kRotThreads);
-        fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
-        mbar_arrive(bar(kBarKRot + s));
-        ++n;
-        it.next();
-      }
+     }
     }
   }
   __syncthreads();

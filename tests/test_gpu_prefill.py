@@ -155,7 +155,7 @@ def full_size_sampled_rows(jl, oracle_mod, name):
         assert torch.equal(out, out0) and torch.equal(lse, lse0)
 
 
-def needle_case(jl, oracle_mod, name, qk_scale=None):
+def needle_case(jl, oracle_mod, name, qk_scale=None, lse_abs=parity.LSE_ABS):
     """Full-size inputs with needles: the needle rows (each dominated by one
     key whose score is right only under the bifocal rule) and 16 seeded rows
     per head.  Besides the gates, the output must be far from the same
@@ -171,7 +171,7 @@ def needle_case(jl, oracle_mod, name, qk_scale=None):
         W.to_oracle_array(q), W.to_oracle_array(k), W.to_oracle_array(v), rb, rq, rh, **kw)
     go, gl = parity.gather_rows(out, lse, rb, rq, rh)
     stats = parity.check(go, gl, ref_o, ref_l, max_abs=parity.BF16_MAX_ABS,
-                         mean_abs=parity.BF16_MEAN_ABS, what=f"{name} needles")
+                         mean_abs=parity.BF16_MEAN_ABS, lse_abs=lse_abs, what=f"{name} needles")
     n = len(nd)
     row_rel = (np.abs(go[:n] - ref_o[:n]).max(axis=1) /
                np.maximum(np.abs(ref_o[:n]).max(axis=1), 1e-30))
@@ -198,8 +198,9 @@ def test_full_size_needles(jl, oracle_mod, name):
 @pytest.mark.parametrize("name", sorted(C.PEAKY))
 def test_full_size_peaky(jl, oracle_mod, name):
     """q and k at four times the configurations' scale (scores with a standard
-    deviation of ~4: a few dozen keys carry each row) plus needles."""
-    needle_case(jl, oracle_mod, name, qk_scale=C.PEAKY[name])
+    deviation of ~4: a few dozen keys carry each row) plus needles; the LSE
+    gate is prefill_cases.PEAKY_LSE_ABS (the reason is stated there)."""
+    needle_case(jl, oracle_mod, name, qk_scale=C.PEAKY[name], lse_abs=C.PEAKY_LSE_ABS)
 
 
 def test_full_size_needles_one_tile_kernel(jl, oracle_mod, monkeypatch):

@@ -53,9 +53,9 @@ def _noalloc(lib, stream, q, kc, vc, pos, cap, B, Hq, Hkv, wl, wp):
 CASES = [
     (1, 32, 8, 20000, 20064, 2048, 4096, 31, 1.0, parity.BF16_MAX_ABS),   # G = 5
     (1, 32, 8, 131071, 131072, 2048, 32768, 32, 1.0, parity.BF16_MAX_ABS),  # G = 4
-    (1, 16, 8, 5000, 5000, 512, 8192, 33, 1.0, parity.BF16_MAX_ABS),      # G = 1, group 2
+    (1, 16, 8, 4999, 5000, 512, 8192, 33, 1.0, parity.BF16_MAX_ABS),      # G = 1, group 2
     (2, 12, 4, 30000, 30016, 0, 8192, 34, 1.0, parity.BF16_MAX_ABS),      # all remote, group 3
-    (1, 8, 2, 40000, 40000, 1000, 16384, 35, 3.0, 0.1),                   # peaked, G = 3
+    (1, 8, 2, 39999, 40000, 1000, 16384, 35, 3.0, 0.1),                   # peaked, G = 3
 ]
 
 
