@@ -81,6 +81,17 @@ enum {
    * cover the whole cache (cache_capacity, or max_pages_per_seq * page_size),
    * so make one call before capturing (it may build or grow the table). */
   JL_FLAG_DEVICE_POS = 1u << 1,
+  /* jl_bifocal_prefill_ex, bf16: rotate the keys once per call instead of in
+   * the attention kernel.  A first pass writes both rotated copies of every
+   * key, R(l) k and R(floor(l / G)) k, into the caller's workspace (at least
+   * jl_bifocal_prefill_rotated_keys_bytes() bytes, 256-byte aligned,
+   * required), and the attention kernel then streams the copy of each pass's
+   * class instead of rotating each K tile in shared memory.  Faster at long
+   * lengths, at the cost of that memory (512 MiB for B = 1, L = 131072,
+   * Hkv = 8, D = 128); the result is the same computation, rounded the same
+   * way up to the order of the fp32 operations that form each rotated key.
+   * Ignored for JL_F32 (that kernel always rotates in place). */
+  JL_FLAG_ROTATE_KEYS_ONCE = 1u << 2,
   /* TEST ONLY (jl_bifocal_decode): exercises the kernels' bounded waits.  The
    * decode kernel's TMA producer withholds its first arrival, so the consumer
    * warps' wait on the first K/V block expires after about one second; they
@@ -121,12 +132,21 @@ jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v,
 size_t jl_bifocal_prefill_workspace_size(int B, int L, int Hkv, int D,
                                          jl_dtype dtype);
 
+/* Bytes of workspace jl_bifocal_prefill_ex needs with JL_FLAG_ROTATE_KEYS_ONCE:
+ * two bf16 copies of the keys, 2 * B * L * Hkv * D * 2 bytes, each rounded up
+ * to 256.  0 for sizes below 1. */
+size_t jl_bifocal_prefill_rotated_keys_bytes(int B, int L, int Hkv, int D);
+
 /*
  * Bifocal prefill with every option.  dtype JL_BF16 (D == 128, tensor cores)
  * or JL_F32 (D in {64, 128}, fp32 CUDA-core kernel; out is fp32).
- * softmax_scale <= 0 selects 1/sqrt(D).  flags: JL_FLAG_NO_BIFOCAL.
- * workspace, workspace_bytes: not used (no workspace is needed); any value,
- * NULL and 0 included, is accepted and nothing is written there.
+ * softmax_scale <= 0 selects 1/sqrt(D).  flags: JL_FLAG_NO_BIFOCAL,
+ * JL_FLAG_ROTATE_KEYS_ONCE.
+ * workspace, workspace_bytes: used only with JL_FLAG_ROTATE_KEYS_ONCE (the
+ * rotated keys; at least jl_bifocal_prefill_rotated_keys_bytes() bytes,
+ * 256-byte aligned, JL_ERR_INVALID_ARG otherwise).  Without the flag no
+ * workspace is needed: any value, NULL and 0 included, is accepted and
+ * nothing is written there.
  */
 jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v,
                                 void *out, float *lse, int B, int L, int Hq,

@@ -14,7 +14,8 @@ import os
 import torch
 
 __all__ = [
-    "NO_BIFOCAL", "DEVICE_POS", "DEBUG_SKIP_ARRIVE", "JetLongError", "group_size", "bifocal_prefill",
+    "NO_BIFOCAL", "DEVICE_POS", "ROTATE_KEYS_ONCE", "DEBUG_SKIP_ARRIVE", "JetLongError", "group_size",
+    "bifocal_prefill", "prefill_rotated_keys_bytes",
     "prefill_workspace_size", "decode_workspace_size", "bifocal_decode",
     "bifocal_prefill_3pass", "prefill_3pass_workspace_size",
     "bifocal_decode_batched", "decode_batched_workspace_size",
@@ -25,6 +26,7 @@ __all__ = [
 
 NO_BIFOCAL = 1 << 0  # JL_FLAG_NO_BIFOCAL
 DEVICE_POS = 1 << 1  # JL_FLAG_DEVICE_POS (set by the bindings when pos is a CUDA tensor)
+ROTATE_KEYS_ONCE = 1 << 2  # JL_FLAG_ROTATE_KEYS_ONCE (prefill: rotated keys in a workspace)
 DEBUG_SKIP_ARRIVE = 1 << 31  # JL_FLAG_DEBUG_SKIP_ARRIVE (tests of the bounded waits only)
 
 _BF16, _F32 = 0, 1
@@ -64,6 +66,8 @@ def load():
     L.jl_bifocal_prefill.argtypes = [p, p, p, p, p, i, i, i, i, i, i, i, d, p]
     L.jl_bifocal_prefill_workspace_size.restype = sz
     L.jl_bifocal_prefill_workspace_size.argtypes = [i, i, i, i, i]
+    L.jl_bifocal_prefill_rotated_keys_bytes.restype = sz
+    L.jl_bifocal_prefill_rotated_keys_bytes.argtypes = [i, i, i, i]
     L.jl_bifocal_prefill_ex.restype = i
     L.jl_bifocal_prefill_ex.argtypes = [p, p, p, p, p, i, i, i, i, i, i, i, d, i,
                                         ctypes.c_float, u, p, sz, p]
@@ -152,10 +156,17 @@ def prefill_workspace_size(B, L, Hkv, D, dtype=torch.bfloat16) -> int:
     return int(load().jl_bifocal_prefill_workspace_size(B, L, Hkv, D, code))
 
 
+def prefill_rotated_keys_bytes(B, L, Hkv, D) -> int:
+    """Workspace bytes of a bf16 prefill with ROTATE_KEYS_ONCE."""
+    return int(load().jl_bifocal_prefill_rotated_keys_bytes(B, L, Hkv, D))
+
+
 def bifocal_prefill(q, k, v, *, w_local, w_pretrained, rope_base, out=None, lse=None,
                     softmax_scale=0.0, flags=0, workspace=None, stream=None):
     """Bifocal causal prefill.  q [B,L,Hq,D], k/v [B,L,Hkv,D] (pre-RoPE),
     bf16 (D=128) or fp32 (D in {64,128}).  Returns (out [B,L,Hq,D], lse [B,Hq,L] fp32).
+    With flags | ROTATE_KEYS_ONCE (bf16) the keys are rotated once into a
+    workspace (allocated here when none is given) instead of in the kernel.
     """
     dtype = q.dtype
     if dtype not in (torch.bfloat16, torch.float32):
@@ -172,6 +183,9 @@ def bifocal_prefill(q, k, v, *, w_local, w_pretrained, rope_base, out=None, lse=
     _need(out, "out", dtype, (B, L, Hq, D))
     _need(lse, "lse", torch.float32, (B, Hq, L))
     ws_ptr, ws_bytes = None, 0
+    if workspace is None and (flags & ROTATE_KEYS_ONCE) and dtype == torch.bfloat16:
+        workspace = torch.empty(prefill_rotated_keys_bytes(B, L, Hkv, D), dtype=torch.uint8,
+                                device=q.device)
     if workspace is not None:
         _need(workspace, "workspace", torch.uint8)
         ws_ptr, ws_bytes = _ptr(workspace), workspace.numel()

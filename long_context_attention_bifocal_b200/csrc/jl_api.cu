@@ -187,6 +187,12 @@ long long jl_group_size(long long L, long long w_pretrained) {
 
 const char *jl_last_error(void) { return g_last_error.c_str(); }
 
+size_t jl_bifocal_prefill_rotated_keys_bytes(int B, int L, int Hkv, int D) {
+  if (B < 1 || L < 1 || Hkv < 1 || D < 1) return 0;
+  const size_t one = static_cast<size_t>(B) * L * Hkv * D * sizeof(__nv_bfloat16);
+  return 2 * ((one + 255) & ~static_cast<size_t>(255));
+}
+
 size_t jl_bifocal_prefill_workspace_size(int B, int L, int Hkv, int D, jl_dtype dtype) {
   // keys are rotated inside the prefill kernels: no workspace for any size
   (void)B, (void)L, (void)Hkv, (void)D, (void)dtype;
@@ -206,7 +212,7 @@ jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v, voi
     return fail(JL_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return fail(JL_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL)) != 0)
+  if ((flags & ~static_cast<unsigned>(JL_FLAG_NO_BIFOCAL | JL_FLAG_ROTATE_KEYS_ONCE)) != 0)
     return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
   if (dtype != JL_BF16 && dtype != JL_F32)
     return fail(JL_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dtype));
@@ -218,7 +224,17 @@ jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v, voi
     return fail(JL_ERR_UNSUPPORTED, "problem too large for one launch");
   if (!(softmax_scale >= 0.f) && !(softmax_scale < 0.f))
     return fail(JL_ERR_INVALID_ARG, "softmax_scale is NaN");
-  (void)workspace, (void)workspace_bytes;  // unused: keys are rotated in the kernels
+  const bool once = dtype == JL_BF16 && (flags & JL_FLAG_ROTATE_KEYS_ONCE);
+  const size_t need_ws = once ? jl_bifocal_prefill_rotated_keys_bytes(B, L, Hkv, D) : 0;
+  if (once) {
+    if (workspace == nullptr)
+      return fail(JL_ERR_INVALID_ARG, "JL_FLAG_ROTATE_KEYS_ONCE needs a workspace");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return fail(JL_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (workspace_bytes < need_ws)
+      return fail(JL_ERR_INVALID_ARG, "workspace too small: %zu bytes, need %zu",
+                  workspace_bytes, need_ws);
+  }
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const long long G = group_size_ll(L, w_pretrained);
@@ -248,6 +264,21 @@ jl_status jl_bifocal_prefill_ex(const void *q, const void *k, const void *v, voi
     return e == cudaSuccess ? JL_OK : cuda_fail(e, "fp32 prefill launch");
   }
 
+  if (once) {
+    // both rotated copies, once, into the workspace; the kernel reads them
+    __nv_bfloat16 *kstd = static_cast<__nv_bfloat16 *>(workspace);
+    __nv_bfloat16 *krem =
+        reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(workspace) + need_ws / 2);
+    const bool need_std = a.w_eff > 0;
+    const bool need_rem = !plain;  // some pair is remote
+    cudaError_t e = launch_rotate_keys(static_cast<const __nv_bfloat16 *>(k),
+                                       need_std ? kstd : nullptr, need_rem ? krem : nullptr,
+                                       a.table, B, L, Hkv, D, a.G, s);
+    if (e != cudaSuccess) return cuda_fail(e, "key rotation launch");
+    a.k = need_std ? kstd : krem;
+    a.k_rem = need_rem ? krem : kstd;
+    a.key_mode = 2;
+  }
   cudaError_t e = launch_attention(a, s);
   return e == cudaSuccess ? JL_OK : cuda_fail(e, "prefill launch");
 }

@@ -37,11 +37,19 @@ int sm_count();
 
 // ---- launchers (each returns the launch's cudaError_t) ----
 cudaError_t launch_rope_table(float2 *cs, int positions, int D, double base, cudaStream_t s);
+// Rotated copies of the keys of a [B,L,Hkv,D] bf16 tensor (the prefill's
+// "rotate the keys once" mode): kstd = R(l) k (if kstd), krem = R(floor(l/G)) k
+// (if krem), same layout.
+cudaError_t launch_rotate_keys(const __nv_bfloat16 *k, __nv_bfloat16 *kstd,
+                               __nv_bfloat16 *krem, RopeTable t, int B, int L,
+                               int Hkv, int D, int G, cudaStream_t s);
 
 struct PrefillArgs {
   const void *q;      // [B,L,Hq,D] pre-RoPE
-  const void *k;      // [B,L,Hkv,D] keys: raw (key_mode 0) or a cache rotated at
-                      // original positions (key_mode 1, batch stride kv_stride)
+  const void *k;      // [B,L,Hkv,D] keys: raw (key_mode 0), a cache rotated at
+                      // original positions (key_mode 1, batch stride kv_stride), or
+                      // rotated at original positions by the library (key_mode 2)
+  const void *k_rem = nullptr;  // key_mode 2: the keys rotated at floor(l / G)
   const void *v;      // [B,L,Hkv,D]
   void *out;          // [B,L,Hq,D]
   float *lse;         // [B,Hq,L]
@@ -55,7 +63,8 @@ struct PrefillArgs {
   int q_off = 0;      // position of query row 0 (multiple of 128); keys are [0, q_off + L)
   int64_t kv_stride = 0;  // keys per batch entry in k and v; 0: q_off + L
   int key_mode = 0;   // 0: raw keys (R(k) / R(f(k)) in the kernel); 1: cached keys at
-                      // original positions (as they are / R(f(k) - k) in the kernel)
+                      // original positions (as they are / R(f(k) - k) in the kernel);
+                      // 2: both rotations done beforehand (k, k_rem read as they are)
 };
 
 cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s);

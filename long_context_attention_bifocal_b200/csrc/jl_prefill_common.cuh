@@ -130,7 +130,10 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8]) {
 // already rotated at their original positions, used as they are by the local
 // passes and moved to f(k) by R(f(k) - k) for the remote ones (techwalker
 // explainer §三: rotations compose, R(a) R(b) = R(a + b)).
-enum : int { kKeysRaw = 0, kKeysCached = 1 };
+// The third mode, kKeysRotated, takes both rotated copies from memory (the
+// opt-in pass that rotates every key once per call): the kernels rotate
+// nothing and read the copy of the pass's class.
+enum : int { kKeysRaw = 0, kKeysCached = 1, kKeysRotated = 2 };
 
 // In-place rotation of part of a 128-key tile in shared memory (bf16, the
 // 128-byte-swizzled K-major layout the TMA wrote: dims 0-63 in the first
@@ -153,6 +156,7 @@ struct KeySlice {
   // they are (cached keys in a local pass)
   static __device__ __forceinline__ int position(int k, int kind, int key_mode, int G) {
     if (key_mode == kKeysRaw) return kind == kStd ? k : k / G;
+    if (key_mode == kKeysRotated) return -1;
     return kind == kStd ? -1 : k - k / G;
   }
 

@@ -124,6 +124,7 @@ struct KParams {
 template <bool kGeneral>
 __global__ void __launch_bounds__(kThreads, 1)
     bifocal_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                 const __grid_constant__ CUtensorMap tm_krem,
                                  const __grid_constant__ CUtensorMap tm_v,
                                  const KParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -401,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------ TMA producer --
       if (lane == 0) {
         prefetch_tmap(&tm_k);
+        if (p.key_mode == kKeysRotated) prefetch_tmap(&tm_krem);
         prefetch_tmap(&tm_v);
         PassIter t;
         t.begin(qt + q_off / kBM, p.w, band);
@@ -412,9 +414,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             raise_abort(abort_s, p.status);
             break;
           }
+          // the raw tile, or with the keys rotated once per call, the copy of
+          // this pass's class
+          const CUtensorMap *km = p.key_mode == kKeysRotated && t.kind() == kRem ? &tm_krem : &tm_k;
           mbar_arrive_expect_tx(bar(kBarKFull + s), kTileBytes);
-          tma_load_4d(sb + kOffK + s * kTileBytes, &tm_k, bar(kBarKFull + s), 0, hk, kBN * t.j, b);
-          tma_load_4d(sb + kOffK + s * kTileBytes + kHalfBytes, &tm_k, bar(kBarKFull + s), 64, hk,
+          tma_load_4d(sb + kOffK + s * kTileBytes, km, bar(kBarKFull + s), 0, hk, kBN * t.j, b);
+          tma_load_4d(sb + kOffK + s * kTileBytes + kHalfBytes, km, bar(kBarKFull + s), 64, hk,
                       kBN * t.j, b);
           ++kiss;
           if (!mbar_wait(bar(kBarVEmpty + s), ph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
@@ -477,7 +482,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ph = (it / kStages) & 1;
           const int sbuf = it & 1;
           const uint32_t sph = (it >> 1) & 1;
-          if (!mbar_wait(bar(kBarKRot + s), ph, abort_s, abort_g, kTimeoutNs) ||
+          // the tile rotated by warps 8-11, or as loaded when the keys were
+          // rotated beforehand
+          if (!mbar_wait(bar((p.key_mode == kKeysRotated ? kBarKFull : kBarKRot) + s), ph, abort_s,
+                         abort_g, kTimeoutNs) ||
               !mbar_wait(bar(kBarSFree + sbuf), sph ^ 1u, abort_s, abort_g, kTimeoutNs)) {
             ok = false;
             break;
@@ -521,7 +529,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       PassIter t;
       t.begin(qt + q_off / kBM, p.w, band);
       int n = 0;
-      while (!t.done()) {
+      // with the keys rotated beforehand there is nothing to do (and nothing
+      // waits for these warps: the MMA warp takes the tiles as loaded)
+      while (p.key_mode != kKeysRotated && !t.done()) {
         const int s = n % kStages;
         const int k0 = kBN * t.j, kind = t.kind();
         // the table read for this tile goes out before the wait for its keys
@@ -590,12 +600,14 @@ cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s) {
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  CUtensorMap mk, mv;
+  CUtensorMap mk, mkr, mv;
   // keys [0, q_off + L); a cache may be longer per batch entry than that
   // (kv_stride keys)
   const int keys = a.q_off + a.L;
   const int64_t kvs = a.kv_stride > 0 ? a.kv_stride : keys;
-  if (!make_map(&mk, a.k, a.B, keys, a.Hkv, kvs) || !make_map(&mv, a.v, a.B, keys, a.Hkv, kvs))
+  if (!make_map(&mk, a.k, a.B, keys, a.Hkv, kvs) ||
+      !make_map(&mkr, a.k_rem ? a.k_rem : a.k, a.B, keys, a.Hkv, kvs) ||
+      !make_map(&mv, a.v, a.B, keys, a.Hkv, kvs))
     return cudaErrorInvalidValue;
   KParams p;
   p.q = static_cast<const __nv_bfloat16 *>(a.q);
@@ -617,9 +629,9 @@ cudaError_t launch_prefill_sm100(const PrefillArgs &a, cudaStream_t s) {
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * a.Hq;
   if (a.band != 0 || a.q_off != 0)
-    bifocal_prefill_sm100_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mv, p);
+    bifocal_prefill_sm100_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
   else
-    bifocal_prefill_sm100_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mv, p);
+    bifocal_prefill_sm100_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
   return cudaGetLastError();
 }
 

@@ -193,6 +193,7 @@ __device__ __forceinline__ void rotate_q_row(uint8_t *dst, int r, const __nv_bfl
 template <bool kGeneral>
 __global__ void __launch_bounds__(kThreads, 1)
     bifocal_prefill_sm100_x2_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                    const __grid_constant__ CUtensorMap tm_krem,
                                     const __grid_constant__ CUtensorMap tm_v,
                                     const KParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -296,8 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       PassIter rit;
       rit.begin(qt + q_off / kBM, p.w, band);
       int rot_n = 0;
+      // with the keys rotated beforehand there is nothing to do: the MMA warp
+      // then waits for the K tiles themselves
+      const bool rotating = p.key_mode != kKeysRotated;
       auto rotate_next = [&]() -> bool {
-        if (rit.done()) return true;
+        if (!rotating || rit.done()) return true;
         const int s = rot_n % kKStages;
         // uniform across the warp, like every wait of the softmax warps
         if (!warp_wait(bar(kBarKFull + s), (rot_n / kKStages) & 1, abort_s, abort_g))
@@ -315,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY, l = 0.f;
       int j = 0;
       while (ok && !it.done()) {
-        if (!rit.done())  // the next slice's table entries, into L1 during the wait
+        if (rotating && !rit.done())  // the next slice's table entries, into L1 during the wait
           ks.prefetch(p.cs, kBN * rit.j, rit.kind(), p.key_mode, p.G, p.n_keys);
         if (!warp_wait(bar(kBarSFull + t), j & 1, abort_s, abort_g)) {
           ok = false;
@@ -506,11 +510,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // n % stages of each.
       if (lane == 0) {
         const bool is_k = warp == kProducerWarp;
-        const CUtensorMap *map = is_k ? &tm_k : &tm_v;
+        const CUtensorMap *vmap = &tm_v;
         const int stages = is_k ? kKStages : kVStages;
         const uint32_t base = sb + (is_k ? kOffK : kOffV);
         const int full = is_k ? kBarKFull : kBarVFull, empty = is_k ? kBarKEmpty : kBarVEmpty;
-        prefetch_tmap(map);
+        prefetch_tmap(is_k ? &tm_k : vmap);
+        if (is_k && p.key_mode == kKeysRotated) prefetch_tmap(&tm_krem);
         PassIter it;
         it.begin(qt + q_off / kBM, p.w, band);
         int n = 0;
@@ -520,6 +525,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             raise_abort(abort_s, p.status);
             break;
           }
+          // K: the raw tile, or with the keys rotated once per call, the copy
+          // of this pass's class
+          const CUtensorMap *map =
+              !is_k ? vmap : (p.key_mode == kKeysRotated && it.kind() == kRem ? &tm_krem : &tm_k);
           mbar_arrive_expect_tx(bar(full + s), kTileBytes);
           tma_load_4d(base + s * kTileBytes, map, bar(full + s), 0, hk, kBN * it.j, b);
           tma_load_4d(base + s * kTileBytes + kHalfBytes, map, bar(full + s), 64, hk, kBN * it.j,
@@ -555,17 +564,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!wait(kBarQReady + t, qphase[t] & 1)) return false;
             ++qphase[t];
           }
-          if (t == 0 && !wait(kBarKRot + s, (jj / kKStages) & 1)) return false;
+          // the tile rotated by the softmax threads, or as loaded when the
+          // keys were rotated beforehand
+          if (t == 0 && !wait((p.key_mode == kKeysRotated ? kBarKFull : kBarKRot) + s,
+                              (jj / kKStages) & 1))
+            return false;
           tc_fence_after();
           const uint32_t a0 = sb + (t == 0 ? kOffQ0 : kOffQ1);
           const uint32_t b0 = sb + kOffK + s * kTileBytes;
-          // a rolled loop: its eight issues take a few tens of cycles against
-          // the product's 512, and it keeps no descriptor live across steps
-#pragma unroll 1
-          for (int kk = 0; kk < 8; ++kk) {
+          auto score_steps = [&](int kk) {
             const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
             umma_bf16(tmem + tm_s(t), sdesc_sw128(a0 + off, 16, 1024),
                       sdesc_sw128(b0 + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          };
+          // Measured on a B200 at L = 131072 (same box, ms per call): issuing
+          // the eight steps as a rolled loop is faster while the softmax
+          // threads rotate the keys (172.5 against 180), the unrolled
+          // sequence when the keys were rotated beforehand (135 against 145).
+          if (p.key_mode == kKeysRotated) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) score_steps(kk);
+          } else {
+#pragma unroll 1
+            for (int kk = 0; kk < 8; ++kk) score_steps(kk);
           }
           umma_commit(bar(kBarSFull + t));
           if (t == 1) umma_commit(bar(kBarKEmpty + s));  // both heads' S issued
@@ -669,12 +690,14 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  CUtensorMap mk, mv;
+  CUtensorMap mk, mkr, mv;
   // keys [0, q_off + L); a cache may be longer per batch entry than that
   // (kv_stride keys)
   const int keys = a.q_off + a.L;
   const int64_t kvs = a.kv_stride > 0 ? a.kv_stride : keys;
-  if (!make_map(&mk, a.k, a.B, keys, a.Hkv, kvs) || !make_map(&mv, a.v, a.B, keys, a.Hkv, kvs))
+  if (!make_map(&mk, a.k, a.B, keys, a.Hkv, kvs) ||
+      !make_map(&mkr, a.k_rem ? a.k_rem : a.k, a.B, keys, a.Hkv, kvs) ||
+      !make_map(&mv, a.v, a.B, keys, a.Hkv, kvs))
     return cudaErrorInvalidValue;
   KParams p;
   p.q = static_cast<const __nv_bfloat16 *>(a.q);
@@ -703,9 +726,9 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * (a.Hq / 2);
   if (a.band != 0 || a.q_off != 0)
-    bifocal_prefill_sm100_x2_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mv, p);
+    bifocal_prefill_sm100_x2_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
   else
-    bifocal_prefill_sm100_x2_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mv, p);
+    bifocal_prefill_sm100_x2_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
   return cudaGetLastError();
 }
 

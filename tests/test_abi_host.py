@@ -85,6 +85,9 @@ INVALID, UNSUPPORTED = 1, 2
     (dict(flags=1 << 7), INVALID),
     (dict(flags=1 << 31), INVALID),       # the decode-only test flag
     (dict(dtype=5), INVALID),
+    (dict(flags=1 << 2), INVALID),                                    # keys rotated once: no workspace
+    (dict(flags=1 << 2, ws=FAKE + 16, ws_bytes=1 << 30), INVALID),    # workspace not 256-aligned
+    (dict(flags=1 << 2, ws=FAKE, ws_bytes=10), INVALID),              # workspace too small
 ])
 def test_prefill_rejects(lib, kw, code):
     assert _prefill(lib, **kw) == code
@@ -124,6 +127,10 @@ def test_workspace_sizes(lib):
     assert lib.jl_bifocal_prefill_workspace_size(1, 131072, 8, 128, 0) == 0
     assert lib.jl_bifocal_prefill_workspace_size(1, 100, 8, 64, 1) == 0
     assert lib.jl_bifocal_prefill_chunk_workspace_size(1, 131072 - 16384, 16384, 8, 128) == 0
+    # the opt-in mode that rotates the keys once: two bf16 copies, 256-aligned each
+    assert lib.jl_bifocal_prefill_rotated_keys_bytes(1, 131072, 8, 128) == 2 * 131072 * 8 * 128 * 2
+    assert lib.jl_bifocal_prefill_rotated_keys_bytes(1, 3, 1, 128) == 2 * 768
+    assert lib.jl_bifocal_prefill_rotated_keys_bytes(0, 3, 1, 128) == 0
     n = lib.jl_bifocal_decode_workspace_size(1, 32, 8, 128, 131071)
     assert n > 0 and n % 4 == 0
     assert lib.jl_bifocal_decode_workspace_size(1, 32, 8, 128, -1) == 0

@@ -75,6 +75,18 @@ def test_bf16_small_all_rows_one_tile_kernel(jl, oracle_mod, case, monkeypatch):
     test_bf16_small_all_rows(jl, oracle_mod, case)
 
 
+@pytest.mark.parametrize("case", SMALL, ids=[C.small_id(c) for c in SMALL])
+def test_bf16_small_keys_rotated_once(jl, oracle_mod, case):
+    """The same cases with the opt-in mode that rotates the keys once per call
+    into a workspace (JL_FLAG_ROTATE_KEYS_ONCE) instead of in the kernel."""
+    q, k, v, kw = C.small_inputs(oracle_mod.default(), case)
+    out, lse = run_prefill(jl, q, k, v, flags=jl.ROTATE_KEYS_ONCE, **kw)
+    ref_o, ref_l = oracle_mod.default().bifocal_all_rows(
+        W.to_oracle_array(q), W.to_oracle_array(k), W.to_oracle_array(v), **kw)
+    parity.check(parity.to_np(out), parity.to_np(lse), ref_o, ref_l,
+                 max_abs=parity.BF16_MAX_ABS, mean_abs=parity.BF16_MEAN_ABS, what=str(case))
+
+
 def test_bf16_explicit_softmax_scale(jl, oracle_mod):
     """A softmax scale given by the caller instead of 1/sqrt(D)."""
     q, k, v = W.prefill_inputs(1, 700, 4, 2, 128, dtype="bf16", value_scale=0.5, seed=12)
@@ -155,7 +167,7 @@ def full_size_sampled_rows(jl, oracle_mod, name):
         assert torch.equal(out, out0) and torch.equal(lse, lse0)
 
 
-def needle_case(jl, oracle_mod, name, qk_scale=None, lse_abs=parity.LSE_ABS):
+def needle_case(jl, oracle_mod, name, qk_scale=None, lse_abs=parity.LSE_ABS, flags=0):
     """Full-size inputs with needles: the needle rows (each dominated by one
     key whose score is right only under the bifocal rule) and 16 seeded rows
     per head.  Besides the gates, the output must be far from the same
@@ -165,7 +177,7 @@ def needle_case(jl, oracle_mod, name, qk_scale=None, lse_abs=parity.LSE_ABS):
     cfg = W.PREFILL[name]
     B, L, Hq = cfg["B"], cfg["L"], cfg["Hq"]
     q, k, v, kw, nd = C.needle_inputs(orc, name, qk_scale=qk_scale)
-    out, lse = run_prefill(jl, q, k, v, **kw)
+    out, lse = run_prefill(jl, q, k, v, flags=flags, **kw)
     rb, rq, rh = C.needle_rows(nd, B, L, Hq, per_head=16, seed=cfg["seed"])
     ref_o, ref_l = orc.bifocal_rows(
         W.to_oracle_array(q), W.to_oracle_array(k), W.to_oracle_array(v), rb, rq, rh, **kw)
@@ -201,6 +213,11 @@ def test_full_size_peaky(jl, oracle_mod, name):
     deviation of ~4: a few dozen keys carry each row) plus needles; the LSE
     gate is prefill_cases.PEAKY_LSE_ABS (the reason is stated there)."""
     needle_case(jl, oracle_mod, name, qk_scale=C.PEAKY[name], lse_abs=C.PEAKY_LSE_ABS)
+
+
+def test_full_size_needles_keys_rotated_once(jl, oracle_mod):
+    """The 8B/128K needle case with the keys rotated once per call."""
+    needle_case(jl, oracle_mod, "qwen3_8b_L131072", flags=jl.ROTATE_KEYS_ONCE)
 
 
 def test_full_size_needles_one_tile_kernel(jl, oracle_mod, monkeypatch):
