@@ -190,7 +190,10 @@ __device__ __forceinline__ void rotate_q_row(uint8_t *dst, int r, const __nv_bfl
 
 // kGeneral: band passes or a query offset (the unfused three-call path and
 // chunked prefill); the default prefill runs the instantiation without them.
-template <bool kGeneral>
+// kRotate: the softmax threads rotate the K tiles (raw or cached keys); false
+// when the keys were rotated once per call beforehand, so that the copy of the
+// loop that reads them carries no rotation code.
+template <bool kGeneral, bool kRotate>
 __global__ void __launch_bounds__(kThreads, 1)
     bifocal_prefill_sm100_x2_kernel(const __grid_constant__ CUtensorMap tm_k,
                                     const __grid_constant__ CUtensorMap tm_krem,
@@ -299,9 +302,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int rot_n = 0;
       // with the keys rotated beforehand there is nothing to do: the MMA warp
       // then waits for the K tiles themselves
-      const bool rotating = p.key_mode != kKeysRotated;
       auto rotate_next = [&]() -> bool {
-        if (!rotating || rit.done()) return true;
+        if (!kRotate || rit.done()) return true;
         const int s = rot_n % kKStages;
         // uniform across the warp, like every wait of the softmax warps
         if (!warp_wait(bar(kBarKFull + s), (rot_n / kKStages) & 1, abort_s, abort_g))
@@ -319,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY, l = 0.f;
       int j = 0;
       while (ok && !it.done()) {
-        if (rotating && !rit.done())  // the next slice's table entries, into L1 during the wait
+        if (kRotate && !rit.done())  // the next slice's table entries, into L1 during the wait
           ks.prefetch(p.cs, kBN * rit.j, rit.kind(), p.key_mode, p.G, p.n_keys);
         if (!warp_wait(bar(kBarSFull + t), j & 1, abort_s, abort_g)) {
           ok = false;
@@ -566,8 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // the tile rotated by the softmax threads, or as loaded when the
           // keys were rotated beforehand
-          if (t == 0 && !wait((p.key_mode == kKeysRotated ? kBarKFull : kBarKRot) + s,
-                              (jj / kKStages) & 1))
+          if (t == 0 && !wait((kRotate ? kBarKRot : kBarKFull) + s, (jj / kKStages) & 1))
             return false;
           tc_fence_after();
           const uint32_t a0 = sb + (t == 0 ? kOffQ0 : kOffQ1);
@@ -581,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the eight steps as a rolled loop is faster while the softmax
           // threads rotate the keys (172.5 against 180), the unrolled
           // sequence when the keys were rotated beforehand (135 against 145).
-          if (p.key_mode == kKeysRotated) {
+          if constexpr (!kRotate) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) score_steps(kk);
           } else {
@@ -683,11 +684,14 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(bifocal_prefill_sm100_x2_kernel<false>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(bifocal_prefill_sm100_x2_kernel<true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    const void *fns[4] = {reinterpret_cast<const void *>(bifocal_prefill_sm100_x2_kernel<false, true>),
+                          reinterpret_cast<const void *>(bifocal_prefill_sm100_x2_kernel<true, true>),
+                          reinterpret_cast<const void *>(bifocal_prefill_sm100_x2_kernel<false, false>),
+                          reinterpret_cast<const void *>(bifocal_prefill_sm100_x2_kernel<true, false>)};
+    for (const void *fn : fns) {
+      if (attr_err == cudaSuccess)
+        attr_err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    }
   });
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap mk, mkr, mv;
@@ -725,10 +729,18 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
   }
   p.scale_log2 = a.scale * 1.4426950408889634f;
   const int64_t grid = static_cast<int64_t>(p.n_qtiles) * a.B * (a.Hq / 2);
-  if (a.band != 0 || a.q_off != 0)
-    bifocal_prefill_sm100_x2_kernel<true><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
-  else
-    bifocal_prefill_sm100_x2_kernel<false><<<static_cast<unsigned>(grid), kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
+  const unsigned g = static_cast<unsigned>(grid);
+  const bool general = a.band != 0 || a.q_off != 0;
+  if (a.key_mode != kKeysRotated) {
+    if (general)
+      bifocal_prefill_sm100_x2_kernel<true, true><<<g, kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
+    else
+      bifocal_prefill_sm100_x2_kernel<false, true><<<g, kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
+  } else if (general) {
+    bifocal_prefill_sm100_x2_kernel<true, false><<<g, kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
+  } else {
+    bifocal_prefill_sm100_x2_kernel<false, false><<<g, kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
+  }
   return cudaGetLastError();
 }
 
