@@ -145,7 +145,9 @@ enum : int { kKeysRaw = 0, kKeysCached = 1, kKeysRotated = 2 };
 // advance by 0 or 1 per key (k, floor(k / G), or k - floor(k / G) for a cache
 // at original positions), so the table is read once, at the first key, and
 // the factors then move on by R(p + 1) = R(p) R(1) (a complex multiplication
-// with row 1 of the table, kept in shared memory as `step`) where p advances.
+// with row 1 of the table, kept in shared memory as `step`: 32 float4, entry
+// 8 e2 + c holding (cos, sin) of theta for pairs 8c + 2 e2 and 8c + 2 e2 + 1)
+// where p advances.
 // All four keys' words are loaded before any is rotated, so one shared-memory
 // latency covers the slice.  Arithmetic in fp32, one rounding to bf16.
 struct KeySlice {
@@ -225,10 +227,13 @@ struct KeySlice {
         // multiples of G; u = k - f everywhere else)
         m = (m + 1 == G) ? 0 : m + 1;
         if (u + 1 < rows && (every || (cached ? (m != 0) : (m == 0)))) {
-          const float4 *st4 = reinterpret_cast<const float4 *>(step + 8 * c);
+          const float4 *st4 = reinterpret_cast<const float4 *>(step);
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
-            const float4 v = st4[e2];  // (cos, sin)(theta) of pairs 2 e2, 2 e2 + 1
+            // (cos, sin)(theta) of pairs 8c + 2 e2, 8c + 2 e2 + 1; the table is
+            // stored e2-major, so the eight chunks of one e2 are 128
+            // contiguous bytes (one conflict-free wavefront for a warp)
+            const float4 v = st4[8 * e2 + c];
             const float c1[2] = {v.x, v.z}, s1[2] = {sg * v.y, sg * v.w};
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -252,14 +257,18 @@ struct KeySlice {
 template <int NTHR>
 struct KeyRotator {
   static constexpr int kRows = kBN * 16 / NTHR;
-  const float4 *step;  // (cos, sin)(theta_i) of the thread's pairs, two per float4
+  // (cos, sin)(theta_i) of the thread's pairs, two per float4: the step table
+  // holds 32 float4, entry q = pairs 4q, 4q + 1 and entry 16 + q = pairs
+  // 4q + 2, 4q + 3, so that sixteen threads' first (or second) halves are 256
+  // contiguous bytes (conflict-free)
+  const float4 *step;
   int i0;              // first pair of this thread
   int kb;              // first key of the thread's block within a tile
 
   __device__ void init(const float2 *step_smem, int tid) {
     i0 = 4 * (tid & 15);
     kb = kRows * (tid >> 4);
-    step = reinterpret_cast<const float4 *>(step_smem + i0);
+    step = reinterpret_cast<const float4 *>(step_smem) + (tid & 15);
   }
 
   struct Start {
@@ -319,7 +328,7 @@ struct KeyRotator {
           make_uint2(sm100::pack_bf16x2(y2[0], y2[1]), sm100::pack_bf16x2(y2[2], y2[3]));
       m = (m + 1 == G) ? 0 : m + 1;
       if (every || (cached ? (m != 0) : (m == 0))) {
-        const float4 t01 = step[0], t23 = step[1];
+        const float4 t01 = step[0], t23 = step[16];
         const float c1[4] = {t01.x, t01.z, t23.x, t23.z};
         const float s1[4] = {t01.y, t01.w, t23.y, t23.w};
 #pragma unroll

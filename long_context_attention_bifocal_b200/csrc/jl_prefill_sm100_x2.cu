@@ -101,7 +101,7 @@ enum : int {
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
 constexpr uint32_t kOffSkip = kOffAbort + 4;
-constexpr uint32_t kOffStep = (kOffSkip + 4 + 15) & ~15u;  // 64 x float2: R(1) per pair
+constexpr uint32_t kOffStep = (kOffSkip + 4 + 15) & ~15u;  // R(1) per pair (32 float4)
 constexpr uint32_t kSmemUsed = kOffStep + 64 * 8;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -252,9 +252,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(sb + kOffTmemSlot, kTmemCols);
     tmem_relinquish();
   }
-  // the key rotation's step factors: table row 1, (cos, sin)(theta_i)
-  if (threadIdx.x < 64)
-    reinterpret_cast<float2 *>(smem + kOffStep)[threadIdx.x] = p.cs[64 + threadIdx.x];
+  // the key rotation's step factors: table row 1, (cos, sin)(theta_i), as
+  // float4 entry 8 e2 + c = pairs 8c + 2 e2 and 8c + 2 e2 + 1
+  if (threadIdx.x < 32) {
+    const int i0 = 8 * (threadIdx.x & 7) + 2 * (threadIdx.x >> 3);
+    const float2 a = p.cs[64 + i0], b2 = p.cs[64 + i0 + 1];
+    reinterpret_cast<float4 *>(smem + kOffStep)[threadIdx.x] = make_float4(a.x, a.y, b2.x, b2.y);
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + kOffTmemSlot);
