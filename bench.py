@@ -41,7 +41,7 @@ PAGE_SIZE = 16  # keys per page of the paged-cache decode line
 # DRAM bytes (read + write) of one full-size launch of the prefill kernel,
 # from ncu (dram__bytes_read.sum + dram__bytes_write.sum, one pass) on B200.
 # Must be re-measured (or set to None) whenever that kernel changes.
-PREFILL_TRAFFIC_BYTES = None
+PREFILL_TRAFFIC_BYTES = 6857217152  # 5.790e9 read + 1.067e9 written, mean of two timed launches
 PREFILL_CFG = "qwen3_8b_L131072"
 DECODE_CFG = "qwen3_8b_decode_n131072"
 
@@ -170,11 +170,16 @@ PREFILL_SWEEP = ["qwen3_1p7b_L65536", "qwen3_4b_L16384", "qwen3_4b_L32768", "qwe
 
 def interleaved(stream, fa, fb, reps):
     """Medians (ms) of fa and fb timed alternately with CUDA events on `stream`
-    (clock drift and neighbours hit both alike)."""
+    (clock drift and neighbours hit both alike).  The stream first runs a
+    ~20 ms wait, so that the host has queued every call before the device
+    reaches the first: the events then time the device work alone, not the
+    host's launch path (which a short decode call would otherwise wait on)."""
     ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(reps)]
     eb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(40_000_000)
     for i, ((a0, a1), (b0, b1)) in enumerate(zip(ea, eb)):
         a0.record(stream)
         fa(i)
@@ -348,6 +353,8 @@ def run_cuda(args):
     def avg_ms(fn, reps):
         es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(reps)]
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(40_000_000)  # the host queues ahead (see interleaved)
         for a, b in es:
             a.record(stream)
             fn()
