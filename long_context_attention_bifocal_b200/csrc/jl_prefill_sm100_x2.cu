@@ -688,10 +688,9 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    const void *fns[4] = {reinterpret_cast<const void *>(bifocal_prefill_sm100_x2_kernel<false, true>),
+    const void *fns[3] = {reinterpret_cast<const void *>(bifocal_prefill_sm100_x2_kernel<false, true>),
                           reinterpret_cast<const void *>(bifocal_prefill_sm100_x2_kernel<true, true>),
-                          reinterpret_cast<const void *>(bifocal_prefill_sm100_x2_kernel<false, false>),
-                          reinterpret_cast<const void *>(bifocal_prefill_sm100_x2_kernel<true, false>)};
+                          reinterpret_cast<const void *>(bifocal_prefill_sm100_x2_kernel<false, false>)};
     for (const void *fn : fns) {
       if (attr_err == cudaSuccess)
         attr_err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
@@ -740,9 +739,10 @@ cudaError_t launch_prefill_sm100_x2(const PrefillArgs &a, cudaStream_t s) {
       bifocal_prefill_sm100_x2_kernel<true, true><<<g, kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
     else
       bifocal_prefill_sm100_x2_kernel<false, true><<<g, kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
-  } else if (general) {
-    bifocal_prefill_sm100_x2_kernel<true, false><<<g, kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
   } else {
+    // keys rotated once per call: only the plain prefill call (no band, no
+    // query offset) takes that mode
+    if (general) return cudaErrorInvalidValue;
     bifocal_prefill_sm100_x2_kernel<false, false><<<g, kThreads, kSmemAlloc, s>>>(mk, mkr, mv, p);
   }
   return cudaGetLastError();
