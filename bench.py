@@ -43,6 +43,7 @@ PAGE_SIZE = 16  # keys per page of the paged-cache decode line
 # Must be re-measured (or set to None) whenever that kernel changes.
 PREFILL_TRAFFIC_BYTES = 6857217152  # 5.790e9 read + 1.067e9 written, mean of two timed launches
 PREFILL_CFG = "qwen3_8b_L131072"
+CPU_ROWS_PER_HEAD = 16  # rows per query head in every timed oracle sample
 DECODE_CFG = "qwen3_8b_decode_n131072"
 
 
@@ -662,7 +663,7 @@ def cpu_baseline(q_h, k_h, v_h, qd_h, kc_h, vc_h, kwp, kwd, pos, budget_s=20.0, 
     orc = oracle.default()
     B, L, Hq, D = q_h.shape
     qa, ka, va = W.to_oracle_array(q_h), W.to_oracle_array(k_h), W.to_oracle_array(v_h)
-    per_head = rows or 16
+    per_head = rows or CPU_ROWS_PER_HEAD
     rb, rq, rh = W.sample_rows(B, L, Hq, per_head=per_head, seed=123)
     t = time.perf_counter()
     orc.bifocal_rows(qa, ka, va, rb, rq, rh, **kwp)
@@ -696,9 +697,10 @@ def run_reference(args):
     kwp = dict(w_local=pc["w_local"], w_pretrained=pc["w_pretrained"], rope_base=pc["rope_base"])
     q, k, v = W.prefill_inputs(B, L, Hq, Hkv, D, value_scale=pc["value_scale"], seed=pc["seed"])
     qa, ka, va = W.to_oracle_array(q), W.to_oracle_array(k), W.to_oracle_array(v)
-    # the oracle runs the rows of one kv head at a time in parallel: give each
-    # kv head at least as many rows as there are host threads
-    per_head = max(2, -(-orc.num_threads() // (Hq // Hkv)))
+    # the same sample size as the in-bench cpu_baseline leg (16 rows per query
+    # head), so that the oracle's per-call work on the whole key sequence is
+    # spread over as many rows and the two CPU figures measure the same thing
+    per_head = CPU_ROWS_PER_HEAD
     times, flops = [], []
     for s in range(args.warmup + args.steps):
         rb, rq, rh = W.sample_rows(B, L, Hq, per_head=per_head, seed=1000 + s)
